@@ -1,0 +1,134 @@
+/*
+ * sigattn.h -- C ABI of the B200 (sm_100a) sigmoid-attention library.
+ *
+ * The library computes bidirectional sigmoid attention over ragged, padded
+ * batches ("Better Models, Faster Training: Sigmoid Attention for single-cell
+ * Foundation Models", sec. 2A):
+ *
+ *     O = sigma(Q K^T / sqrt(d) + b) V,   sigma(x) = 1/(1+e^-x),   b = -ln(n_b)
+ *
+ * and its gradient with respect to Q, K and V (sec. 2B: sigma' = sigma(1-sigma);
+ * sec. 2C: one kernel for dQ and one for dK/dV, activations recomputed, no
+ * atomics). n_b is the valid length of sequence b; tokens at positions >= n_b
+ * are padding and are ignored on both the query and the key side (sec. 2C,
+ * native padding support): P_ij = 0 unless i < n_b and j < n_b.
+ *
+ * Conventions shared by every call
+ *  - Tensors Q, K, V, dO, O, dQ, dK, dV are bf16, contiguous [B][H][Lmax][d]
+ *    (d fastest), in device memory, 16-byte aligned. d must be 64 or 128.
+ *  - lengths is int32 [B] in device memory; each n_b must lie in [0, Lmax].
+ *    A value outside that range is treated as 0 (all outputs of sequence b
+ *    are zero) and raises SIGATTN_ERR_INVALID_ARG in the workspace's sticky
+ *    error word (read it with sigattn_read_error).
+ *  - Outputs are fully written: rows i >= n_b of O, dQ, dK and dV are exact
+ *    zeros. Values in padded rows of the inputs are never used, but must be
+ *    finite: a padded value v enters as 0 * v inside the tensor-core sums.
+ *  - The scale is 1/sqrt(d) and the bias -ln(n_b) is computed in-kernel; the
+ *    bias has no gradient. There is no causal mask.
+ *  - Arithmetic: bf16 operands, fp32 accumulation, P (and dS) rounded to bf16
+ *    before the second matrix product, outputs rounded to nearest bf16.
+ *  - workspace: caller-owned device memory of at least
+ *    sigattn_workspace_size(B, H, Lmax, d) bytes, 16-byte aligned. Each call
+ *    writes its work list there; calls that may run concurrently (different
+ *    streams) need different workspaces. Word 0 is a sticky error status, so
+ *    zero the workspace once after allocating it (cudaMemset); the library
+ *    keeps it consistent afterwards.
+ *  - stream: a cudaStream_t (NULL = legacy default stream). Calls only
+ *    enqueue work: they neither allocate nor synchronise.
+ *  - Return value: a sigattn_status. Argument errors are reported before
+ *    anything is enqueued. A kernel-side timeout (a bounded wait that gave up)
+ *    is recorded in the workspace and surfaces through sigattn_read_error.
+ *  - Ownership: the library keeps no pointer after a call returns.
+ */
+#ifndef SIGATTN_H_
+#define SIGATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SIGATTN_API __attribute__((visibility("default")))
+#else
+#define SIGATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SIGATTN_OK = 0,
+  SIGATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad length */
+  SIGATTN_ERR_UNSUPPORTED = 2, /* d not in {64, 128}, or a size beyond the limits */
+  SIGATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  SIGATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (sticky, in the workspace) */
+} sigattn_status;
+
+/* Work-list kinds (used by the plan helpers). */
+enum { SIGATTN_KIND_FWD = 0, SIGATTN_KIND_DQ = 1, SIGATTN_KIND_DKDV = 2 };
+
+/* Limits: 1 <= B <= SIGATTN_MAX_BATCH, 1 <= H, 1 <= Lmax <= SIGATTN_MAX_LEN. */
+#define SIGATTN_MAX_BATCH 4096
+#define SIGATTN_MAX_LEN (1 << 20)
+
+/* Library version, e.g. 100 for 0.1.0. */
+SIGATTN_API int sigattn_version(void);
+
+/* Human-readable name of a status code (static string). */
+SIGATTN_API const char* sigattn_status_str(int status);
+
+/* Rows of one work item for a kind: 256 (forward), 128 (dQ), 128 (dK/dV).
+ * Returns -1 for an unknown kind. */
+SIGATTN_API int sigattn_block_rows(int kind);
+
+/* Bytes of workspace needed for any of the three calls with these sizes
+ * (a 256-byte header plus one 8-byte entry per possible work item).
+ * Returns 0 if the sizes are out of range. */
+SIGATTN_API size_t sigattn_workspace_size(int B, int H, int Lmax, int d);
+
+/* Forward pass (sec. 2A): o = sigma(q k^T / sqrt(d) - ln n) v.
+ * q, k, v: inputs; o: output. All [B][H][Lmax][d] bf16 on the device. */
+SIGATTN_API int sigattn_fwd(const void* q, const void* k, const void* v, void* o, const int32_t* lengths, int B, int H,
+                int Lmax, int d, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward pass, query side (sec. 2B/2C): dq = (1/sqrt(d)) * dS k with
+ * dS = (dout v^T) * P * (1 - P). dout is the gradient of the loss w.r.t. o. */
+SIGATTN_API int sigattn_bwd_dq(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                   const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* Backward pass, key/value side (sec. 2B/2C): dk = (1/sqrt(d)) * dS^T q and
+ * dv = P^T dout. */
+SIGATTN_API int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                     const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* Run only the ragged tile scheduler for `kind` on the device: afterwards the
+ * workspace holds, at byte offset 8, the item count (int32), and at byte
+ * offset 256, `count` pairs (int32 bh = b*H + h, int32 block index), ordered
+ * longest sequence first (ties in batch order), heads ascending, blocks
+ * ascending. Only blocks whose first row is < n_b appear (sec. 2C: fully
+ * padded blocks are skipped). */
+SIGATTN_API int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/* Host-side statement of the same schedule (no GPU needed): writes up to
+ * `cap` (bh, block) pairs to `items_out` (2*cap int32) and the full count to
+ * `*count`. lengths_host is host memory. */
+SIGATTN_API int sigattn_plan_host(const int32_t* lengths_host, int B, int H, int Lmax, int kind, int32_t* items_out, int cap,
+                      int* count);
+
+/* Text of the last CUDA failure behind a SIGATTN_ERR_CUDA returned to the
+ * calling thread (static, thread-local; "no error" if none yet). */
+SIGATTN_API const char* sigattn_last_error(void);
+
+/* Synchronise `stream`, read the workspace's sticky error word, clear it and
+ * return it (SIGATTN_OK if no kernel reported a problem). If `site` is not
+ * NULL it receives a code naming the failing check or wait (0 if none). */
+SIGATTN_API int sigattn_read_error(void* workspace, int* site, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIGATTN_H_ */

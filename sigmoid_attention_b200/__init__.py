@@ -1,0 +1,238 @@
+"""Python binding of the B200 sigmoid-attention C ABI (``include/sigattn.h``).
+
+Argument marshalling only: each ``sigattn_*`` function here passes device
+pointers, sizes and the current CUDA stream to the function of the same name
+in ``libsigattn.so``; every step of the computation runs in the library's CUDA
+kernels. PyTorch provides device memory and streams. There is no fallback: if
+the library is missing or a call fails, an exception is raised.
+
+The library computes O = sigma(Q K^T / sqrt(d) - ln n) V over padded
+[B, H, Lmax, d] bf16 batches with per-sequence valid lengths n, and the
+gradients dQ, dK, dV ("Better Models, Faster Training: Sigmoid Attention for
+single-cell Foundation Models", sec. 2A-2C).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "SigattnError", "library", "library_path", "sigattn_version", "sigattn_status_str", "sigattn_block_rows",
+    "sigattn_workspace_size", "sigattn_fwd", "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
+    "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "read_plan", "make_workspace", "forward", "backward",
+    "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
+]
+
+KIND_FWD, KIND_DQ, KIND_DKDV = 0, 1, 2
+STATUS = {0: "SIGATTN_OK", 1: "SIGATTN_ERR_INVALID_ARG", 2: "SIGATTN_ERR_UNSUPPORTED", 3: "SIGATTN_ERR_CUDA",
+          4: "SIGATTN_ERR_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsigattn.so")
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+
+class SigattnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library():
+    """Load ``libsigattn.so`` (built in-tree by ``sigmoid_attention_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: run `python -m sigmoid_attention_b200.build` first")
+        lib = ctypes.CDLL(_LIB_PATH)
+        lib.sigattn_version.restype = _i
+        lib.sigattn_version.argtypes = []
+        lib.sigattn_status_str.restype = ctypes.c_char_p
+        lib.sigattn_status_str.argtypes = [_i]
+        lib.sigattn_block_rows.restype = _i
+        lib.sigattn_block_rows.argtypes = [_i]
+        lib.sigattn_workspace_size.restype = _sz
+        lib.sigattn_workspace_size.argtypes = [_i] * 4
+        lib.sigattn_fwd.restype = _i
+        lib.sigattn_fwd.argtypes = [_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp]
+        lib.sigattn_bwd_dq.restype = _i
+        lib.sigattn_bwd_dq.argtypes = [_vp] * 6 + [_i] * 4 + [_vp, _sz, _vp]
+        lib.sigattn_bwd_dkdv.restype = _i
+        lib.sigattn_bwd_dkdv.argtypes = [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]
+        lib.sigattn_plan.restype = _i
+        lib.sigattn_plan.argtypes = [_vp] + [_i] * 5 + [_vp, _sz, _vp]
+        lib.sigattn_plan_host.restype = _i
+        lib.sigattn_plan_host.argtypes = [_vp] + [_i] * 4 + [_vp, _i, ctypes.POINTER(_i)]
+        lib.sigattn_last_error.restype = ctypes.c_char_p
+        lib.sigattn_last_error.argtypes = []
+        lib.sigattn_read_error.restype = _i
+        lib.sigattn_read_error.argtypes = [_vp, ctypes.POINTER(_i), _vp]
+        _lib = lib
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        err = SigattnError(fn, status)
+        if status == 3:
+            err.args = (f"{err.args[0]} ({library().sigattn_last_error().decode()})",)
+        raise err
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dims(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected a [B, H, Lmax, d] tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=torch.bfloat16) -> int:
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    return t.data_ptr()
+
+
+def sigattn_version() -> int:
+    return library().sigattn_version()
+
+
+def sigattn_status_str(status: int) -> str:
+    return library().sigattn_status_str(status).decode()
+
+
+def sigattn_block_rows(kind: int) -> int:
+    return library().sigattn_block_rows(kind)
+
+
+def sigattn_workspace_size(B: int, H: int, Lmax: int, d: int) -> int:
+    return library().sigattn_workspace_size(B, H, Lmax, d)
+
+
+def make_workspace(B: int, H: int, Lmax: int, d: int, device=None) -> torch.Tensor:
+    """A zero-initialised workspace (uint8 CUDA tensor) big enough for any call."""
+    n = sigattn_workspace_size(B, H, Lmax, d)
+    if n == 0:
+        raise SigattnError("sigattn_workspace_size", 2)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sigattn_fwd(q, k, v, o, lengths, workspace, stream=None) -> None:
+    B, H, L, d = _dims(q)
+    _check("sigattn_fwd", library().sigattn_fwd(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lengths, "lengths", torch.int32),
+        B, H, L, d, _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_bwd_dq(q, k, v, dout, dq, lengths, workspace, stream=None) -> None:
+    B, H, L, d = _dims(q)
+    _check("sigattn_bwd_dq", library().sigattn_bwd_dq(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dq, "dq"),
+        _dev(lengths, "lengths", torch.int32), B, H, L, d, _dev(workspace, "workspace", torch.uint8),
+        workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_bwd_dkdv(q, k, v, dout, dk, dv, lengths, workspace, stream=None) -> None:
+    B, H, L, d = _dims(q)
+    _check("sigattn_bwd_dkdv", library().sigattn_bwd_dkdv(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dk, "dk"), _dev(dv, "dv"),
+        _dev(lengths, "lengths", torch.int32), B, H, L, d, _dev(workspace, "workspace", torch.uint8),
+        workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_plan(lengths, B, H, Lmax, d, kind, workspace, stream=None) -> None:
+    _check("sigattn_plan", library().sigattn_plan(
+        _dev(lengths, "lengths", torch.int32), B, H, Lmax, d, kind, _dev(workspace, "workspace", torch.uint8),
+        workspace.numel(), _stream_ptr(stream)))
+
+
+def read_plan(workspace: torch.Tensor) -> torch.Tensor:
+    """The (bh, block) pairs the last plan wrote, as an int32 CPU tensor [count, 2]."""
+    words = workspace.view(torch.int32).cpu()
+    count = int(words[2])
+    return words[64:64 + 2 * count].view(count, 2).clone()
+
+
+def sigattn_plan_host(lengths, H: int, Lmax: int, kind: int) -> torch.Tensor:
+    """Host statement of the schedule: int32 [count, 2] of (bh, block) pairs."""
+    lens = torch.as_tensor(lengths, dtype=torch.int32).contiguous()
+    B = lens.numel()
+    count = ctypes.c_int(0)
+    lib = library()
+    _check("sigattn_plan_host", lib.sigattn_plan_host(lens.data_ptr(), B, H, Lmax, kind, None, 0,
+                                                      ctypes.byref(count)))
+    out = torch.zeros(max(count.value, 1), 2, dtype=torch.int32)
+    _check("sigattn_plan_host", lib.sigattn_plan_host(lens.data_ptr(), B, H, Lmax, kind, out.data_ptr(),
+                                                      count.value, ctypes.byref(count)))
+    return out[:count.value]
+
+
+def sigattn_last_error() -> str:
+    return library().sigattn_last_error().decode()
+
+
+def sigattn_read_error(workspace, stream=None):
+    """Synchronise, read and clear the workspace's sticky error word: (status, site)."""
+    site = ctypes.c_int(0)
+    st = library().sigattn_read_error(_dev(workspace, "workspace", torch.uint8), ctypes.byref(site),
+                                      _stream_ptr(stream))
+    return st, site.value
+
+
+# ---------------------------------------------------------------------------
+# Convenience wrappers (allocate outputs with torch, then call the C ABI)
+# ---------------------------------------------------------------------------
+def forward(q, k, v, lengths, workspace=None, stream=None) -> torch.Tensor:
+    B, H, L, d = _dims(q)
+    if workspace is None:
+        workspace = make_workspace(B, H, L, d, q.device)
+    o = torch.empty_like(q)
+    sigattn_fwd(q, k, v, o, lengths, workspace, stream)
+    return o
+
+
+def backward(q, k, v, dout, lengths, workspace=None, stream=None):
+    B, H, L, d = _dims(q)
+    if workspace is None:
+        workspace = make_workspace(B, H, L, d, q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    sigattn_bwd_dq(q, k, v, dout, dq, lengths, workspace, stream)
+    sigattn_bwd_dkdv(q, k, v, dout, dk, dv, lengths, workspace, stream)
+    return dq, dk, dv
+
+
+class SigmoidAttentionFunction(torch.autograd.Function):
+    """Autograd wrapper: forward with ``sigattn_fwd``, backward with the two
+    backward calls (a drop-in for softmax attention over padded batches)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, lengths):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        ws = make_workspace(*_dims(q), q.device)
+        o = forward(q, k, v, lengths, ws)
+        ctx.save_for_backward(q, k, v, lengths, ws)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, lengths, ws = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, do.contiguous(), lengths, ws)
+        return dq, dk, dv, None
+
+
+def sigmoid_attention(q, k, v, lengths) -> torch.Tensor:
+    return SigmoidAttentionFunction.apply(q, k, v, lengths)

@@ -1,0 +1,245 @@
+// api.cu -- the C ABI (include/sigattn.h): argument checks, TMA tensor maps and
+// the launches of the plan and compute kernels. No allocation, no host sync
+// (except in sigattn_read_error, which exists to synchronise).
+#include <climits>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sigattn.h"
+#include "common.cuh"
+
+namespace sigattn {
+cudaError_t launch_prep(const int* lengths, int B, int H, int L, int d, int kind, int* ws, void* out0, void* out1,
+                        int num_sms, cudaStream_t stream);
+int plan_host(const int* lengths, int B, int H, int L, int kind, int* out, int cap);
+cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                       const int* lengths, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                          const CUtensorMap& tv, void* dq, const int* lengths, int* ws, int B, int H, int L,
+                          int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_dkdv(int d, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                            const CUtensorMap& tdo, void* dk, void* dv, const int* lengths, int* ws, int B, int H,
+                            int L, int num_sms, cudaStream_t stream);
+}  // namespace sigattn
+
+using namespace sigattn;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  int num_sms = 0;
+  bool supported = false;
+};
+
+// SM count and architecture check of the current device (cached per device).
+bool device_info(DeviceInfo* out) {
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!have[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    cache[dev].num_sms = sms;
+    cache[dev].supported = (major == 10 && minor == 0);
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  return true;
+}
+
+// 3-D view {d, Lmax, B*H} of a [B][H][Lmax][d] bf16 tensor, loaded as
+// [128 rows][64 columns] boxes with the 128-byte swizzle the tcgen05
+// descriptors expect. Rows past Lmax read as zeros.
+bool make_map(CUtensorMap* map, const void* ptr, int BH, int L, int d) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+long long max_items(int B, int H, int L) {
+  return static_cast<long long>(B) * H * ceil_div(L, kBwdItemRows);
+}
+
+int check_sizes(int B, int H, int L, int d) {
+  if (d != 64 && d != 128) return SIGATTN_ERR_UNSUPPORTED;
+  if (B < 1 || H < 1 || L < 1) return SIGATTN_ERR_INVALID_ARG;
+  if (B > kMaxBatch || L > kMaxLen) return SIGATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > INT_MAX / 2 || max_items(B, H, L) > INT_MAX / 4)
+    return SIGATTN_ERR_UNSUPPORTED;
+  return SIGATTN_OK;
+}
+
+// Text of the last CUDA failure seen by this thread (see sigattn_last_error).
+thread_local char g_last_error[160] = "no error";
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SIGATTN_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return SIGATTN_ERR_CUDA;
+}
+
+int map_failure() {
+  snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed or is unavailable");
+  return SIGATTN_ERR_CUDA;
+}
+
+int check_call(int B, int H, int L, int d, const int32_t* lengths, const void* ws, size_t ws_bytes,
+               DeviceInfo* info) {
+  int st = check_sizes(B, H, L, d);
+  if (st != SIGATTN_OK) return st;
+  if (lengths == nullptr || (reinterpret_cast<uintptr_t>(lengths) & 3u) != 0) return SIGATTN_ERR_INVALID_ARG;
+  if (!aligned16(ws) || ws_bytes < sigattn_workspace_size(B, H, L, d)) return SIGATTN_ERR_INVALID_ARG;
+  if (!device_info(info)) {
+    const cudaError_t e = cudaGetLastError();
+    return cuda_status(e != cudaSuccess ? e : cudaErrorUnknown);
+  }
+  if (!info->supported) return SIGATTN_ERR_UNSUPPORTED;
+  return SIGATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sigattn_version(void) { return 100; }
+
+const char* sigattn_status_str(int status) {
+  switch (status) {
+    case SIGATTN_OK: return "ok";
+    case SIGATTN_ERR_INVALID_ARG: return "invalid argument";
+    case SIGATTN_ERR_UNSUPPORTED: return "unsupported size or device";
+    case SIGATTN_ERR_CUDA: return "CUDA error";
+    case SIGATTN_ERR_TIMEOUT: return "kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int sigattn_block_rows(int kind) {
+  if (kind < SIGATTN_KIND_FWD || kind > SIGATTN_KIND_DKDV) return -1;
+  return item_rows(kind);
+}
+
+size_t sigattn_workspace_size(int B, int H, int Lmax, int d) {
+  if (check_sizes(B, H, Lmax, d) != SIGATTN_OK) return 0;
+  return static_cast<size_t>(kHeaderWords) * 4 + static_cast<size_t>(max_items(B, H, Lmax)) * 8;
+}
+
+int sigattn_fwd(const void* q, const void* k, const void* v, void* o, const int32_t* lengths, int B, int H,
+                int Lmax, int d, void* workspace, size_t workspace_bytes, void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SIGATTN_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) || !make_map(&tv, v, B * H, Lmax, d))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(lengths, B, H, Lmax, d, SIGATTN_KIND_FWD, ws, o, nullptr, info.num_sms, s));
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(launch_fwd(d, tq, tk, tv, o, lengths, ws, B, H, Lmax, info.num_sms, s));
+}
+
+int sigattn_bwd_dq(const void* q, const void* k, const void* v, const void* dout, void* dq, const int32_t* lengths,
+                   int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes, void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq))
+    return SIGATTN_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) ||
+      !make_map(&tv, v, B * H, Lmax, d) || !make_map(&tdo, dout, B * H, Lmax, d))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(lengths, B, H, Lmax, d, SIGATTN_KIND_DQ, ws, dq, nullptr, info.num_sms, s));
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(launch_bwd_dq(d, tq, tdo, tk, tv, dq, lengths, ws, B, H, Lmax, info.num_sms, s));
+}
+
+int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                     const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
+    return SIGATTN_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) ||
+      !make_map(&tv, v, B * H, Lmax, d) || !make_map(&tdo, dout, B * H, Lmax, d))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(lengths, B, H, Lmax, d, SIGATTN_KIND_DKDV, ws, dk, dv, info.num_sms, s));
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(launch_bwd_dkdv(d, tk, tv, tq, tdo, dk, dv, lengths, ws, B, H, Lmax, info.num_sms, s));
+}
+
+int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  if (kind < SIGATTN_KIND_FWD || kind > SIGATTN_KIND_DKDV) return SIGATTN_ERR_INVALID_ARG;
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(launch_prep(lengths, B, H, Lmax, d, kind, static_cast<int*>(workspace), nullptr, nullptr,
+                                 info.num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+int sigattn_plan_host(const int32_t* lengths_host, int B, int H, int Lmax, int kind, int32_t* items_out, int cap,
+                      int* count) {
+  if (kind < SIGATTN_KIND_FWD || kind > SIGATTN_KIND_DKDV) return SIGATTN_ERR_INVALID_ARG;
+  if (lengths_host == nullptr || count == nullptr || cap < 0 || (cap > 0 && items_out == nullptr))
+    return SIGATTN_ERR_INVALID_ARG;
+  const int st = check_sizes(B, H, Lmax, 64);
+  if (st != SIGATTN_OK) return st;
+  *count = plan_host(lengths_host, B, H, Lmax, kind, items_out, cap);
+  return SIGATTN_OK;
+}
+
+const char* sigattn_last_error(void) { return g_last_error; }
+
+int sigattn_read_error(void* workspace, int* site, void* stream) {
+  if (!aligned16(workspace)) return SIGATTN_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int hdr[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(hdr), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (site) *site = hdr[kHdrErrorSite];
+  return hdr[kHdrError];
+}
+
+}  // extern "C"

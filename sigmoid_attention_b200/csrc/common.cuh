@@ -1,0 +1,77 @@
+// common.cuh -- constants and small device helpers shared by the plan, forward
+// and backward kernels of the sigmoid-attention library.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace sigattn {
+
+// Rows of one work item, per call kind. A work item is one block of
+// consecutive rows of one (batch, head) slice holding >= 1 valid token:
+//  * forward: 256 query rows (two 128-row query tiles sharing each K/V block),
+//  * dQ:      128 query rows,
+//  * dK/dV:   128 key rows.
+// Every inner loop walks blocks of 128 columns (keys for forward/dQ, queries
+// for dK/dV) up to ceil(n/128), so fully padded blocks are never touched on
+// either side.
+enum Kind : int { kKindFwd = 0, kKindDq = 1, kKindDkdv = 2 };
+constexpr int kFwdItemRows = 256;
+constexpr int kBwdItemRows = 128;
+constexpr int kColBlock = 128;
+constexpr int kMaxBatch = 4096;        // sequences per call (plan runs in one CTA)
+constexpr int kMaxLen = 1 << 20;       // Lmax bound (TMA coordinates are int32)
+
+__host__ __device__ constexpr int item_rows(int kind) { return kind == kKindFwd ? kFwdItemRows : kBwdItemRows; }
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Valid length of sequence b, or 0 if the caller's value is outside [0, L]
+// (the plan flags that case in the workspace header).
+__device__ __forceinline__ int load_len(const int* lengths, int b, int L) {
+  const int n = __ldg(lengths + b);
+  return (n < 0 || n > L) ? 0 : n;
+}
+
+struct Item {
+  int bh;   // b * H + h
+  int blk;  // row-block index within the slice
+};
+
+__device__ __forceinline__ Item load_item(const int* ws, int idx) {
+  const int2 v = reinterpret_cast<const int2*>(ws + kHeaderWords)[idx];
+  return Item{v.x, v.y};
+}
+
+// 1/sqrt(d) for the supported head sizes.
+template <int D>
+struct Scale;
+template <>
+struct Scale<64> {
+  static constexpr float value = 0.125f;
+};
+template <>
+struct Scale<128> {
+  static constexpr float value = 0.08838834764831845f;
+};
+
+// sigma(s * scale + bias) for one score, written as 1/2 + tanh(x/2)/2 with the
+// hardware tanh ("a hardware-optimised tanh approximation for the sigmoid",
+// Better Models, Faster Training, sec. 2C). half_scale = scale/2 and
+// half_bias = bias/2 are folded into one FMA.
+__device__ __forceinline__ float sigmoid_from_score(float s, float half_scale, float half_bias) {
+  const float t = tanh_approx(fmaf(s, half_scale, half_bias));
+  return fmaf(t, 0.5f, 0.5f);
+}
+
+// Store `D` bf16 zeros at `dst` (16-byte aligned, D a multiple of 8).
+template <int D>
+__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst) {
+  uint4* p = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) p[i] = make_uint4(0, 0, 0, 0);
+}
+
+}  // namespace sigattn

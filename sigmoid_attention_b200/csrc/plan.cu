@@ -1,0 +1,152 @@
+// plan.cu -- the ragged tile scheduler and padded-row zero fill.
+//
+// "Native padding support": blocks that hold only padding are skipped on both
+// the query and the key side (Better Models, Faster Training: Sigmoid
+// Attention for single-cell Foundation Models, sec. 2C). Here that becomes a
+// work list built on the device from the per-sequence valid lengths, so the
+// host never has to read the lengths back:
+//
+//   * one work item per (b, h, row block) whose first row is < n_b; the
+//     compute kernels walk column blocks only up to ceil(n_b / 128);
+//   * sequences are ordered longest first (stable in b), and a persistent
+//     compute grid takes items round-robin, which spreads the long items over
+//     all SMs first (longest-processing-time-first order);
+//   * rows of the outputs that no item covers (rows >= ceil(n_b/rows)*rows)
+//     are written as exact zeros by the same launch, so padded rows of every
+//     output are 0 without a separate memset.
+#include <algorithm>
+#include <numeric>
+#include <vector>
+
+#include "common.cuh"
+
+namespace sigattn {
+
+__global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ lengths, int B, int H, int L, int d,
+                                                    int rows, int* __restrict__ ws, __nv_bfloat16* out0,
+                                                    __nv_bfloat16* out1) {
+  extern __shared__ int smem_plan[];
+  const int tid = threadIdx.x;
+
+  if (blockIdx.x == 0) {
+    int* s_len = smem_plan;            // [B]
+    int* s_order = smem_plan + B;      // [B]
+    int* s_off = smem_plan + 2 * B;    // [B + 1]
+    for (int b = tid; b < B; b += blockDim.x) {
+      const int n = __ldg(lengths + b);
+      if (n < 0 || n > L) {
+        atomicCAS(ws + kHdrError, 0, 1 /* SIGATTN_ERR_INVALID_ARG */);
+        atomicExch(ws + kHdrErrorSite, -(b + 1));
+      }
+      s_len[b] = (n < 0 || n > L) ? 0 : n;
+    }
+    __syncthreads();
+    // Rank of each sequence in the longest-first order (ties keep batch order).
+    for (int b = tid; b < B; b += blockDim.x) {
+      const int nb = s_len[b];
+      int rank = 0;
+      for (int o = 0; o < B; ++o) {
+        const int no = s_len[o];
+        rank += (no > nb) || (no == nb && o < b);
+      }
+      s_order[rank] = b;
+    }
+    __syncthreads();
+    if (tid == 0) s_off[0] = 0;
+    for (int s = tid; s < B; s += blockDim.x) s_off[s + 1] = H * ceil_div(s_len[s_order[s]], rows);
+    __syncthreads();
+    // Inclusive scan of s_off[1..B] by warp 0, 32 entries at a time.
+    if (tid < 32) {
+      int carry = 0;
+      for (int base = 0; base < B; base += 32) {
+        const int i = base + tid;
+        int v = (i < B) ? s_off[i + 1] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (tid >= o) v += u;
+        }
+        v += carry;
+        if (i < B) s_off[i + 1] = v;
+        carry = __shfl_sync(0xffffffffu, v, 31);
+      }
+    }
+    __syncthreads();
+    const int total = s_off[B];
+    if (tid == 0) ws[kHdrCount] = total;
+    int2* items = reinterpret_cast<int2*>(ws + kHeaderWords);
+    for (int i = tid; i < total; i += blockDim.x) {
+      int lo = 0, hi = B - 1;  // find s with s_off[s] <= i < s_off[s + 1]
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= i) lo = mid; else hi = mid - 1;
+      }
+      const int b = s_order[lo];
+      const int local = i - s_off[lo];
+      const int nblk = ceil_div(s_len[b], rows);
+      items[i] = make_int2(b * H + local / nblk, local % nblk);
+    }
+  }
+
+  // Zero the rows no work item covers, in every output.
+  if (out0 == nullptr) return;
+  const int chunks_per_row = d / 8;  // 16-byte chunks
+  for (int slice = blockIdx.x; slice < B * H; slice += gridDim.x) {
+    const int b = slice / H;
+    const int n = load_len(lengths, b, L);
+    const int cover = min(L, ceil_div(n, rows) * rows);
+    const long long nchunks = static_cast<long long>(L - cover) * chunks_per_row;
+    const size_t base = (static_cast<size_t>(slice) * L + cover) * d;
+    uint4* p0 = reinterpret_cast<uint4*>(out0 + base);
+    uint4* p1 = out1 ? reinterpret_cast<uint4*>(out1 + base) : nullptr;
+    for (long long c = tid; c < nchunks; c += blockDim.x) {
+      p0[c] = make_uint4(0, 0, 0, 0);
+      if (p1) p1[c] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+cudaError_t launch_prep(const int* lengths, int B, int H, int L, int d, int kind, int* ws, void* out0,
+                        void* out1, int num_sms, cudaStream_t stream) {
+  const int smem = (3 * B + 1) * static_cast<int>(sizeof(int));
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (3 * kMaxBatch + 1) * static_cast<int>(sizeof(int)));
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int grid = std::max(1, std::min(B * H, 2 * num_sms));
+  prep_kernel<<<grid, 1024, smem, stream>>>(lengths, B, H, L, d, item_rows(kind), ws,
+                                            static_cast<__nv_bfloat16*>(out0),
+                                            static_cast<__nv_bfloat16*>(out1));
+  return cudaGetLastError();
+}
+
+// Host restatement of the same schedule (used by the host-side tests and for
+// debugging): items in the order the device plan writes them.
+int plan_host(const int* lengths, int B, int H, int L, int kind, int* out, int cap) {
+  const int rows = item_rows(kind);
+  std::vector<int> len(B), order(B);
+  for (int b = 0; b < B; ++b) len[b] = (lengths[b] < 0 || lengths[b] > L) ? 0 : lengths[b];
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return len[a] > len[b]; });
+  int count = 0;
+  for (int s = 0; s < B; ++s) {
+    const int b = order[s];
+    const int nblk = ceil_div(len[b], rows);
+    for (int h = 0; h < H; ++h)
+      for (int m = 0; m < nblk; ++m) {
+        if (count < cap) {
+          out[2 * count] = b * H + h;
+          out[2 * count + 1] = m;
+        }
+        ++count;
+      }
+  }
+  return count;
+}
+
+}  // namespace sigattn

@@ -1,0 +1,190 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Tolerances, all against fp64 on the same bf16 inputs:
+  O:           rel-L2 <= 5e-3 and max-abs <= 2e-2
+  dQ, dK, dV:  rel-L2 <= 1e-2
+  active-tile list, zeros in padded rows, run-to-run results: bit-exact.
+Small cases compare every element; the full-size workloads compare sampled
+rows computed one by one by the oracle, plus properties checked everywhere.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sigmoid_attention_b200 as sa
+from sigmoid_attention_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+FWD_REL, FWD_ABS, BWD_REL = 5e-3, 2e-2, 1e-2
+
+
+def rel_l2(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    return np.linalg.norm(got - ref) / max(den, 1e-300)
+
+
+def run_gpu(q, k, v, dout, lengths):
+    dev = torch.device("cuda")
+    B, H, L, d = q.shape
+    qd, kd, vd, dod = (t.to(dev).contiguous() for t in (q, k, v, dout))
+    lens = torch.as_tensor(lengths, dtype=torch.int32).to(dev)
+    ws = sa.make_workspace(B, H, L, d, dev)
+    o = torch.full_like(qd, float("nan"))  # poison: every element must be written
+    dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
+    sa.sigattn_fwd(qd, kd, vd, o, lens, ws)
+    sa.sigattn_bwd_dq(qd, kd, vd, dod, dq, lens, ws)
+    sa.sigattn_bwd_dkdv(qd, kd, vd, dod, dk, dv, lens, ws)
+    st, site = sa.sigattn_read_error(ws)
+    assert st == 0, (st, site)
+    return [t.float().cpu() for t in (o, dq, dk, dv)]
+
+
+def check_padded_zero(t, lengths):
+    for b, n in enumerate(np.asarray(lengths)):
+        pad = t[b, :, int(n):]
+        assert torch.equal(pad, torch.zeros_like(pad)), f"padded rows of sequence {b} not exactly zero"
+
+
+def check_full(q, k, v, dout, lengths):
+    o, dq, dk, dv = run_gpu(q, k, v, dout, lengths)
+    for t in (o, dq, dk, dv):
+        assert torch.isfinite(t).all()
+        check_padded_zero(t, lengths)
+    o_ref = oracle.forward(q, k, v, lengths)
+    dq_ref, dk_ref, dv_ref = oracle.backward(q, k, v, dout, lengths)
+    assert rel_l2(o, o_ref) <= FWD_REL, rel_l2(o, o_ref)
+    assert np.abs(o.numpy() - o_ref).max() <= FWD_ABS
+    for name, got, ref in (("dq", dq, dq_ref), ("dk", dk, dk_ref), ("dv", dv, dv_ref)):
+        assert rel_l2(got, ref) <= BWD_REL, (name, rel_l2(got, ref))
+    return o, dq, dk, dv
+
+
+SMALL_CASES = [
+    # (B, H, L, d, lengths, seed)
+    (2, 2, 64, 64, [37, 64], 1001),                       # the tiny workload
+    (4, 2, 700, 64, [700, 129, 1, 0], 11),                # several tiles, ragged tail, n=1, n=0
+    (3, 2, 520, 128, [520, 256, 255], 12),
+    (8, 1, 300, 64, [1, 127, 128, 129, 255, 256, 257, 300], 13),   # block edges
+    (8, 1, 300, 128, [1, 127, 128, 129, 255, 256, 257, 300], 14),
+    (2, 3, 200, 128, [200, 77], 15),                      # Lmax not a multiple of 128
+    (1, 2, 1024, 64, [1024], 16),                         # unpadded, several 256-row items
+]
+
+
+@pytest.mark.parametrize("B,H,L,d,lengths,seed", SMALL_CASES)
+def test_small_cases_elementwise(B, H, L, d, lengths, seed):
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, seed)
+    check_full(q, k, v, dout, lengths)
+
+
+def test_tiny_workload_closed_form_zero_query():
+    # Q = 0: every valid weight is 1/(1+n), so O_i = sum_{j<n} V_j / (1+n).
+    B, H, L, d = 2, 2, 64, 64
+    _, k, v, dout = workloads.make_inputs(B, H, L, d, 77)
+    q = torch.zeros_like(k)
+    o, *_ = run_gpu(q, k, v, dout, [37, 64])
+    for b, n in enumerate([37, 64]):
+        expect = v[b, :, :n].double().sum(dim=1, keepdim=True) / (1 + n)
+        assert rel_l2(o[b, :, :n], expect.expand(-1, n, -1)) <= FWD_REL
+
+
+def test_padded_inputs_are_ignored_bitwise():
+    B, H, L, d = 3, 2, 300, 64
+    lens = [300, 140, 17]
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 21)
+    base = run_gpu(q, k, v, dout, lens)
+    q2, k2, v2, do2 = (t.clone() for t in (q, k, v, dout))
+    g = torch.Generator().manual_seed(5)
+    for b, n in enumerate(lens):
+        for t in (q2, k2, v2, do2):
+            t[b, :, n:] = (100 * torch.randn(t[b, :, n:].shape, generator=g)).to(t.dtype)
+    other = run_gpu(q2, k2, v2, do2, lens)
+    for a, b_ in zip(base, other):
+        assert torch.equal(a, b_)
+
+
+def test_deterministic_bitwise():
+    B, H, L, d = 2, 4, 640, 128
+    lens = [640, 333]
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 22)
+    a = run_gpu(q, k, v, dout, lens)
+    b = run_gpu(q, k, v, dout, lens)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("kind", [0, 1, 2])
+def test_device_plan_bit_exact(kind):
+    H, L, d = 3, 1000, 64
+    lens_np = np.array([0, 1, 127, 128, 129, 255, 256, 257, 999, 1000, 513, 640], dtype=np.int32)
+    lens = torch.from_numpy(lens_np).cuda()
+    ws = sa.make_workspace(len(lens_np), H, L, d)
+    sa.sigattn_plan(lens, len(lens_np), H, L, d, kind, ws)
+    torch.cuda.synchronize()
+    dev_items = sa.read_plan(ws)
+    host_items = sa.sigattn_plan_host(lens_np, H, L, kind)
+    assert torch.equal(dev_items, host_items)  # same list, same order
+    got = sorted((int(bh) // H, int(bh) % H, int(m)) for bh, m in dev_items.tolist())
+    expect = [tuple(t) for t in oracle.tiles(lens_np, H, L, sa.sigattn_block_rows(kind)).tolist()]
+    assert got == expect
+
+
+def test_invalid_length_flags_error_and_zeros_sequence():
+    B, H, L, d = 2, 1, 64, 64
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 23)
+    dev = torch.device("cuda")
+    lens = torch.tensor([70, 64], dtype=torch.int32, device=dev)   # 70 > Lmax
+    ws = sa.make_workspace(B, H, L, d, dev)
+    o = torch.full((B, H, L, d), float("nan"), dtype=torch.bfloat16, device=dev)
+    sa.sigattn_fwd(q.to(dev), k.to(dev), v.to(dev), o, lens, ws)
+    st, site = sa.sigattn_read_error(ws)
+    assert st == 1 and site == -1
+    assert torch.equal(o[0].float().cpu(), torch.zeros(H, L, d))
+    o_ref = oracle.forward(q[1:], k[1:], v[1:], [64])
+    assert rel_l2(o[1:].float().cpu(), o_ref) <= FWD_REL
+    assert sa.sigattn_read_error(ws)[0] == 0  # cleared by the read
+
+
+def _sampled(w, nsamp=48, seed=0):
+    q, k, v, dout, lens = workloads.workload_inputs(w)
+    o, dq, dk, dv = run_gpu(q, k, v, dout, lens.numpy())
+    for t in (o, dq, dk, dv):
+        assert torch.isfinite(t).all()
+        check_padded_zero(t, lens.numpy())
+    rng = np.random.default_rng(seed)
+    bh = rng.integers(0, w.B * w.H, nsamp)
+    # sample valid rows, including each sequence's last valid row
+    n_of = lens.numpy()[bh // w.H]
+    row = np.where(rng.random(nsamp) < 0.2, n_of - 1, (rng.random(nsamp) * n_of).astype(np.int64))
+    keep = n_of > 0
+    bh, row = bh[keep], row[keep]
+    for name, got, tol in (("o", o, FWD_REL), ("dq", dq, BWD_REL), ("dk", dk, BWD_REL), ("dv", dv, BWD_REL)):
+        ref = oracle.rows(name, q, k, v, dout, lens.numpy(), bh, row)
+        g = got.reshape(w.B * w.H, w.L, w.d)[bh, row].numpy()
+        assert rel_l2(g, ref) <= tol, (w.name, name, rel_l2(g, ref))
+        if name == "o":
+            assert np.abs(g - ref).max() <= FWD_ABS
+
+
+@pytest.mark.parametrize("name", ["scrna_ragged", "dense_d128", "long_8k", "pad_sweep_p00", "pad_sweep_p25",
+                                  "pad_sweep_p50", "pad_sweep_p75"])
+def test_full_size_workloads_sampled(name):
+    _sampled(workloads.WORKLOADS[name])
+
+
+def test_autograd_function_matches_direct_calls():
+    B, H, L, d = 2, 2, 256, 64
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 31)
+    lens = torch.tensor([256, 100], dtype=torch.int32, device="cuda")
+    qd, kd, vd = (t.cuda().requires_grad_(True) for t in (q, k, v))
+    o = sa.sigmoid_attention(qd, kd, vd, lens)
+    o.backward(dout.cuda())
+    ref_o, ref_dq, ref_dk, ref_dv = run_gpu(q, k, v, dout, [256, 100])
+    assert torch.equal(o.detach().float().cpu(), ref_o)
+    assert torch.equal(qd.grad.float().cpu(), ref_dq)
+    assert torch.equal(kd.grad.float().cpu(), ref_dk)
+    assert torch.equal(vd.grad.float().cpu(), ref_dv)
