@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the sigmoid-attention library on B200.
+
+One step = one pass of the whole hot path over one batch: the forward call and
+both backward calls (dQ, then dK/dV), each of which runs the ragged plan and
+its compute kernel. The headline value counts valid-token FLOPs only
+(4*d per valid (i, j) pair forward + 10*d backward, the usual five-product
+count) divided by the device time of the timed steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run, one process per GPU) every rank
+runs its own batch of the same workload: the (b, h) slices are independent, so
+the work shards with no collective on the data path (weak scaling). Rank 0
+prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sigmoid-attn fwd & bwd TFLOPS (valid tokens) on 1 B200; % of BF16 tensor peak"
+L2_BYTES = 126 * 1024 * 1024
+# Matrix-product FLOPs each call performs per valid (i, j) pair, in units of d:
+# forward S and PV; dQ kernel S, dP, dQ; dK/dV kernel S, dP, dV, dK.
+KERNEL_FLOPS_PER_PAIR = {"fwd": 4, "bwd_dq": 6, "bwd_dkdv": 8}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"bf16_tflops": float(p["bf16_tflops"]), "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]),
+                "hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def _csrc_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sigmoid_attention_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel: str, workload: str, launches_scale: float = 1.0):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    when the summary was taken on other kernel sources or another workload."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("csrc_hash") != _csrc_hash():
+        return None
+    entry = t.get("kernels", {}).get(kernel, {}).get(workload)
+    if not entry:
+        return None
+    return float(entry["dram_bytes_per_launch"]) * launches_scale
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[2:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, max_seconds: float) -> float:
+    """Units all ranks processed divided by the slowest rank's time."""
+    return flops_per_rank * world / max_seconds / 1e12
+
+
+def cpu_baseline(w, target_s: float = 12.0):
+    """The fp64 oracle, as it stands, on the host cores: forward + backward of
+    whole (b, h) slices of the workload's first sequence, as many heads as fit
+    in about `target_s` seconds (at least one)."""
+    import oracle
+    from sigmoid_attention_b200 import workloads
+
+    q, k, v, dout = workloads.make_inputs(1, w.H, w.L, w.d, w.seed)
+    n = int(w.lengths()[0])
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    done_heads, spent = 0, 0.0
+    while done_heads < w.H and (done_heads == 0 or spent * (done_heads + 1) / done_heads <= target_s):
+        sl = slice(done_heads, done_heads + 1)
+        t0 = time.perf_counter()
+        oracle.forward(q[:, sl], k[:, sl], v[:, sl], [n])
+        oracle.backward(q[:, sl], k[:, sl], v[:, sl], dout[:, sl], [n])
+        spent += time.perf_counter() - t0
+        done_heads += 1
+    flops = 14.0 * w.d * n * n * done_heads
+    return {"value": flops / spent / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{done_heads} (b,h) slice(s) of sequence 0 (n={n}, d={w.d}), fwd+bwd in fp64, "
+                      f"{spent:.1f} s"}
+
+
+def run_reference(args, w):
+    """The reference arm: the oracle timed on the host cores (rank 0 only)."""
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from sigmoid_attention_b200 import workloads
+
+    q, k, v, dout = workloads.make_inputs(1, 1, w.L, w.d, w.seed)
+    n = int(w.lengths()[0])
+    # One step = forward + backward of one (b, h) slice, shortened to m query
+    # rows and m key rows when a full slice would not fit the time budget.
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    m0 = min(n, 512)
+    t0 = time.perf_counter()
+    oracle.forward(q[..., :m0, :], k[..., :m0, :], v[..., :m0, :], [m0])
+    oracle.backward(q[..., :m0, :], k[..., :m0, :], v[..., :m0, :], dout[..., :m0, :], [m0])
+    per_pair = (time.perf_counter() - t0) / (m0 * m0)
+    m = n
+    while m > 64 and per_pair * m * m > budget:
+        m //= 2
+    qs, ks, vs, ds = (t[:, :, :m].contiguous() for t in (q, k, v, dout))
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.forward(qs, ks, vs, [m])
+        oracle.backward(qs, ks, vs, ds, [m])
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = float(np.mean(times))
+    flops = 14.0 * w.d * m * m
+    value = flops / sec / 1e12
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    sample = f"one (b,h) slice of sequence 0 cut to {m} of its {n} tokens, fwd+bwd in fp64"
+    line = {"metric": METRIC, "value": value, "unit": "TFLOPS", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {**w.describe(), "step": "oracle fwd+bwd of a bounded sample"},
+            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gpu(args, w):
+    import torch
+
+    import sigmoid_attention_b200 as sa
+    from sigmoid_attention_b200 import workloads
+
+    world, rank, local = _dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    q, k, v, dout, lengths = workloads.workload_inputs(w)
+    flops_fwd = w.fwd_flops()
+    flops_bwd = w.bwd_flops()
+    pairs = flops_fwd / (4.0 * w.d)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, dout))
+    lens = lengths.to(dev)
+    o, dq, dk, dv = (torch.empty_like(qd) for _ in range(4))
+    ws = sa.make_workspace(w.B, w.H, w.L, w.d, dev)
+    stream = torch.cuda.current_stream(dev)
+    tensor_bytes = qd.numel() * 2
+    footprint = 8 * tensor_bytes
+    flush = footprint < 4 * L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sa.sigattn_fwd(qd, kd, vd, o, lens, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        sa.sigattn_bwd_dq(qd, kd, vd, dod, dq, lens, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        sa.sigattn_bwd_dkdv(qd, kd, vd, dod, dk, dv, lens, ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+        if flush:
+            scratch.zero_()
+    st, site = sa.sigattn_read_error(ws, stream)
+    if st != 0:
+        raise SystemExit(f"kernel reported status {st} at site {site}")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            step(events[i])
+            if flush:
+                scratch.zero_()
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    per_kernel = {"fwd": [], "bwd_dq": [], "bwd_dkdv": []}
+    step_ms = []
+    for ev in events:
+        per_kernel["fwd"].append(ev[0].elapsed_time(ev[1]))
+        per_kernel["bwd_dq"].append(ev[1].elapsed_time(ev[2]))
+        per_kernel["bwd_dkdv"].append(ev[2].elapsed_time(ev[3]))
+        step_ms.append(ev[0].elapsed_time(ev[3]))
+    st, site = sa.sigattn_read_error(ws, stream)
+    if st != 0:
+        raise SystemExit(f"kernel reported status {st} at site {site}")
+    total_s = reduce_max(sum(step_ms) / 1e3, world, dev)
+    fwd_s = reduce_max(sum(per_kernel["fwd"]) / 1e3, world, dev)
+    bwd_s = reduce_max((sum(per_kernel["bwd_dq"]) + sum(per_kernel["bwd_dkdv"])) / 1e3, world, dev)
+    value = whole_job_tflops((flops_fwd + flops_bwd) * args.steps, world, total_s)
+    fwd_tflops = whole_job_tflops(flops_fwd * args.steps, world, fwd_s)
+    bwd_tflops = whole_job_tflops(flops_bwd * args.steps, world, bwd_s)
+
+    # --- end to end through the public API with host buffers -------------
+    pin = [t.pin_memory() for t in (q, k, v, dout)]
+    lens_h = lengths.pin_memory()
+    outs_h = [torch.empty_like(q).pin_memory() for _ in range(4)]
+    h2d = sum(t.numel() * t.element_size() for t in pin) + lens_h.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        for src, dst in zip(pin, (qd, kd, vd, dod)):
+            dst.copy_(src, non_blocking=True)
+        lens.copy_(lens_h, non_blocking=True)
+        step()
+        for src, dst in zip((o, dq, dk, dv), outs_h):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = reduce_max(e0.elapsed_time(e1) / 1e3, world, dev)
+    e2e_value = whole_job_tflops((flops_fwd + flops_bwd) * e2e_steps, world, e2e_s)
+
+    peaks = _peaks()
+    peak = peaks["bf16_tflops"]
+    avg_ms = {kname: float(np.mean(v_)) for kname, v_ in per_kernel.items()}
+    dominant = max(avg_ms, key=avg_ms.get)
+    dom_flops = KERNEL_FLOPS_PER_PAIR[dominant] * w.d * pairs
+    achieved = dom_flops / (avg_ms[dominant] / 1e3) / 1e12
+    kernels = {kname: {"ms": avg_ms[kname],
+                       "tflops": KERNEL_FLOPS_PER_PAIR[kname] * w.d * pairs / (avg_ms[kname] / 1e3) / 1e12,
+                       "flops_per_valid_pair": f"{KERNEL_FLOPS_PER_PAIR[kname]}*d"} for kname in avg_ms}
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_s * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**w.describe(), "valid_pairs_per_head": pairs / w.H,
+                   "step": "sigattn_fwd + sigattn_bwd_dq + sigattn_bwd_dkdv (each: plan + compute kernel)",
+                   "flops": "valid pairs only: 4*d fwd + 10*d bwd per pair",
+                   "parallelism": f"replica per GPU x{world} (independent batches)",
+                   "l2": ("flushed between steps (footprint %.0f MB)" % (footprint / 1e6)) if flush else
+                         ("no flush: inputs+outputs %.0f MB > 126 MB L2" % (footprint / 1e6))},
+        "fwd_tflops": fwd_tflops, "bwd_tflops": bwd_tflops,
+        "fwd_frac_of_peak": fwd_tflops / peak, "bwd_frac_of_peak": bwd_tflops / peak,
+        "frac_of_spec_2250": {"fwd": fwd_tflops / 2250.0, "bwd": bwd_tflops / 2250.0},
+        "kernels": kernels,
+        "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": f"bf16_tflops ({peaks['source']}, burst)",
+                     "traffic": _traffic(dominant, w.name)},
+        "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    from sigmoid_attention_b200 import workloads
+
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="dense_d128", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = workloads.WORKLOADS[args.workload]
+    world, _, _ = _dist_env()
+    if world != args.gpus:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
