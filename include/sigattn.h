@@ -118,6 +118,32 @@ SIGATTN_API int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int
 SIGATTN_API int sigattn_plan_host(const int32_t* lengths_host, int B, int H, int Lmax, int kind, int32_t* items_out, int cap,
                       int* count);
 
+/* Size of the fixed device scratch array used by sigattn_fwd_noalloc. */
+#define SIGATTN_NOALLOC_SCRATCH_BYTES (1 << 20)
+
+/* sigattn_fwd for callers that cannot allocate device memory (code that runs
+ * where cudaMalloc is unavailable or forbidden, e.g. inside a host framework
+ * that owns the whole device pool, or a plugin that may only touch the
+ * buffers it is handed). The paper has no counterpart: it is a deployment
+ * convenience of this library.
+ *  - Same computation, inputs and outputs as sigattn_fwd; instead of a
+ *    caller workspace it uses a SIGATTN_NOALLOC_SCRATCH_BYTES array that is
+ *    part of the library's device image, held on every GPU that loads the
+ *    library until the process exits. It calls no cudaMalloc/cudaFree.
+ *  - Size limit: sigattn_workspace_size(B, H, Lmax, d) must not exceed
+ *    SIGATTN_NOALLOC_SCRATCH_BYTES, i.e. B*H*ceil(Lmax/128) <= 131040 work
+ *    items; larger problems return SIGATTN_ERR_UNSUPPORTED (message in
+ *    sigattn_last_error) before anything is enqueued.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call, on every stream, shares the one array: calls that overlap
+ *    on the GPU race. Each call clears the array's status words first.
+ *  - status_out: optional device int32; if not NULL, receives (in stream
+ *    order) this call's device-side status: 0, SIGATTN_ERR_INVALID_ARG for an
+ *    out-of-range length, or SIGATTN_ERR_TIMEOUT. */
+SIGATTN_API int sigattn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, const int32_t* lengths,
+                                    int B, int H, int Lmax, int d, int32_t* status_out, void* stream);
+
 /* Text of the last CUDA failure behind a SIGATTN_ERR_CUDA returned to the
  * calling thread (static, thread-local; "no error" if none yet). */
 SIGATTN_API const char* sigattn_last_error(void);

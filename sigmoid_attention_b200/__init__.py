@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "SigattnError", "library", "library_path", "sigattn_version", "sigattn_status_str", "sigattn_block_rows",
-    "sigattn_workspace_size", "sigattn_fwd", "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
+    "sigattn_workspace_size", "sigattn_fwd", "sigattn_fwd_noalloc", "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
     "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "read_plan", "make_workspace", "forward", "backward",
     "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
 ]
@@ -73,6 +73,8 @@ def library():
         lib.sigattn_plan.argtypes = [_vp] + [_i] * 5 + [_vp, _sz, _vp]
         lib.sigattn_plan_host.restype = _i
         lib.sigattn_plan_host.argtypes = [_vp] + [_i] * 4 + [_vp, _i, ctypes.POINTER(_i)]
+        lib.sigattn_fwd_noalloc.restype = _i
+        lib.sigattn_fwd_noalloc.argtypes = [_vp] * 5 + [_i] * 4 + [_vp, _vp]
         lib.sigattn_last_error.restype = ctypes.c_char_p
         lib.sigattn_last_error.argtypes = []
         lib.sigattn_read_error.restype = _i
@@ -84,7 +86,7 @@ def library():
 def _check(fn: str, status: int) -> None:
     if status != 0:
         err = SigattnError(fn, status)
-        if status == 3:
+        if status in (2, 3):
             err.args = (f"{err.args[0]} ({library().sigattn_last_error().decode()})",)
         raise err
 
@@ -136,6 +138,16 @@ def sigattn_fwd(q, k, v, o, lengths, workspace, stream=None) -> None:
     _check("sigattn_fwd", library().sigattn_fwd(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lengths, "lengths", torch.int32),
         B, H, L, d, _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_fwd_noalloc(q, k, v, o, lengths, status_out=None, stream=None) -> None:
+    """Forward pass without a workspace, for callers that cannot allocate
+    device memory: the library's own fixed scratch array is used instead."""
+    B, H, L, d = _dims(q)
+    st_ptr = _dev(status_out, "status_out", torch.int32) if status_out is not None else None
+    _check("sigattn_fwd_noalloc", library().sigattn_fwd_noalloc(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lengths, "lengths", torch.int32),
+        B, H, L, d, st_ptr, _stream_ptr(stream)))
 
 
 def sigattn_bwd_dq(q, k, v, dout, dq, lengths, workspace, stream=None) -> None:

@@ -21,6 +21,7 @@ cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tdo, 
 cudaError_t launch_bwd_dkdv(int d, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                             const CUtensorMap& tdo, void* dk, void* dv, const int* lengths, int* ws, int B, int H,
                             int L, int num_sms, cudaStream_t stream);
+void set_last_error(const char* msg);
 }  // namespace sigattn
 
 using namespace sigattn;
@@ -106,6 +107,12 @@ int cuda_status(cudaError_t e) {
   snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
   return SIGATTN_ERR_CUDA;
 }
+
+}  // namespace
+
+void sigattn::set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
+namespace {
 
 int map_failure() {
   snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed or is unavailable");
