@@ -56,6 +56,14 @@ bool device_info(DeviceInfo* out) {
   static bool have[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  // A thread that has not used this library's CUDA runtime yet (for example
+  // torch's autograd worker) may have no current context, which the tensor-map
+  // encoder needs; cudaSetDevice makes the device's primary context current.
+  thread_local int ready_for = -1;
+  if (ready_for != dev) {
+    if (cudaSetDevice(dev) != cudaSuccess) return false;
+    ready_for = dev;
+  }
   if (!have[dev]) {
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;

@@ -18,15 +18,27 @@
 //   dK/dV(KV=1) keys    K  V  |        Q   dO | K Q^T    V dO^T    A1 += dS^T Q    -> dK
 //                                                                   A2 += P^T dO    -> dV
 //
-// Each 128-column block is processed as two 64-column halves g = 0, 1, one
-// per epilogue warpgroup, so that the tensor core computes one half while the
-// other half's epilogue runs:
-//   S_g  = R1 C1[g]^T, dP_g = R2 C2[g]^T       (tcgen05.mma, both operands in smem)
-//   epilogue g: P = sigma(S*scale + b) (0 for padded columns), dS = dP P (1-P),
-//               written back as bf16 into the first 32 columns of S_g / dP_g
-//   A1 += dS_g C1[g], A2 += P_g C2[g]          (tcgen05.mma with A read from TMEM)
-// Warps: 0-3 epilogue half 0, 4-7 epilogue half 1, 8 TMA producer, 9 MMA.
-// TMEM: S_g at 64g, dP_g at 128 + 64g, A1 at 256, A2 at 256 + D.
+// Per 128-column block j, in tensor memory (TMEM):
+//   XS  = R1 C1_j^T  (S,  fp32)  -> epilogue: P = sigma(S*scale + b), 0 for
+//                                   padded columns; bf16 P to its own region
+//   XdP = R2 C2_j^T  (dP, fp32)  -> epilogue: dS = dP P (1 - P); bf16 dS to
+//                                   its own region
+//   A1 += dS C1_j, A2 += P C2_j  (A operand read from TMEM, per 32-column chunk)
+// A region is released as soon as the epilogue has copied it to registers, so
+// the products of block j+1 overlap the epilogue of block j. S comes first:
+// P, and with it the dV products and the release of C2, are ready before dP.
+// One thread issues a tcgen05.mma only every ~100 cycles, so the products are
+// spread over several issuing warps: S, dP (when they have separate TMEM
+// regions), A1 and A2. C1 and C2 have rings of their own: C2 (V for dQ, dO
+// for dK/dV) is released earlier than C1, so C1 gets the deeper ring.
+//
+// TMEM columns (512): with separate S and dP regions (dQ, and dK/dV at D=64):
+//   XS [0,128) XdP [128,256) P [256,320) dS [320,384) A1 [384,384+D) A2 after;
+// dK/dV at D=128 has room for one region X [0,128) that holds S, then dP:
+//   X [0,128) P [128,192) dS [192,256) A1 [256,384) A2 [384,512).
+// Warps: 0-7 epilogue (0-3: columns 0-63, 4-7: columns 64-127), 8 TMA
+// producer, then the issuers: S (owns TMEM), dP (separate regions only), A1,
+// A2 (dK/dV only).
 #include "common.cuh"
 
 namespace sigattn {
@@ -35,78 +47,95 @@ template <int D, bool KV>
 struct BwdCfg {
   static constexpr int BM = kBwdItemRows;   // 128 rows per item
   static constexpr int BN = kColBlock;      // 128 columns per block
-  static constexpr int ST = (D == 128) ? 2 : 3;
+  static constexpr bool SPLIT_X = !(KV && D == 128);
+  static constexpr int ST1 = (D == 128) ? 3 : 4;   // C1 ring slots
+  static constexpr int ST2 = (D == 128) ? 2 : 4;   // C2 ring slots
   static constexpr int BOX_BYTES = 128 * 64 * 2;
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int OFF_R1 = 0;
   static constexpr int OFF_R2 = TILE_BYTES;
-  static constexpr int OFF_C = 2 * TILE_BYTES;  // stage s: C1 at OFF_C + 2s*TILE, C2 right after
-  static constexpr int SMEM_BYTES = OFF_C + ST * 2 * TILE_BYTES;
+  static constexpr int OFF_C1 = 2 * TILE_BYTES;
+  static constexpr int OFF_C2 = OFF_C1 + ST1 * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_C2 + ST2 * TILE_BYTES;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-  static constexpr int TM_S = 0;
-  static constexpr int TM_DP = 128;
-  static constexpr int TM_A1 = 256;
-  static constexpr int TM_A2 = 256 + D;
+  static constexpr int TM_XS = 0;
+  static constexpr int TM_XDP = SPLIT_X ? 128 : 0;
+  static constexpr int TM_P = SPLIT_X ? 256 : 128;
+  static constexpr int TM_DS = TM_P + 64;
+  static constexpr int TM_A1 = TM_DS + 64;
+  static constexpr int TM_A2 = TM_A1 + D;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static_assert(TM_A1 + (KV ? 2 : 1) * D <= TMEM_COLS, "TMEM budget");
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int ISSUERS = 2 + (SPLIT_X ? 1 : 0) + (KV ? 1 : 0);
+  static constexpr int THREADS = (EPI_WARPS + 1 + ISSUERS) * 32;
+  // Load both dP chunks at once when registers allow (fewer warps).
+  static constexpr bool DP_BOTH = THREADS <= 384;
 };
 
-template <int ST>
+template <int ST1, int ST2>
 struct BwdBarriers {
   uint64_t r_full, r_empty;
-  uint64_t c_full[ST], c_empty[ST];
-  uint64_t s_full[2], p_full[2];
+  uint64_t c1_full[ST1], c1_empty[ST1];
+  uint64_t c2_full[ST2], c2_empty[ST2];
+  uint64_t xs_full, xdp_full;      // S / dP of the current block are in TMEM
+  uint64_t xs_read, xdp_read;      // the epilogue has copied S / dP out
+  uint64_t p_full[4], ds_full[4];  // bf16 P / dS of a 32-column chunk written
+  uint64_t p_free, ds_free;        // the accumulation products of a block have read P / dS
   uint64_t acc_full, acc_empty;
-  uint64_t drain;
+  uint64_t drain[4];
   uint32_t tmem_base;
   int abort;
 };
 
-// Convert 32 fp32 accumulator values (times `mul`) to bf16 and store them.
-__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul) {
-  uint4* p = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    p[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q + 0]) * mul, __uint_as_float(v[8 * q + 1]) * mul),
-                      pack_bf16x2(__uint_as_float(v[8 * q + 2]) * mul, __uint_as_float(v[8 * q + 3]) * mul),
-                      pack_bf16x2(__uint_as_float(v[8 * q + 4]) * mul, __uint_as_float(v[8 * q + 5]) * mul),
-                      pack_bf16x2(__uint_as_float(v[8 * q + 6]) * mul, __uint_as_float(v[8 * q + 7]) * mul));
-  }
-}
-
-__device__ __forceinline__ void store_zero32(__nv_bfloat16* dst) {
-  uint4* p = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) p[q] = make_uint4(0, 0, 0, 0);
-}
-
 template <int D, bool KV>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_r1, const __grid_constant__ CUtensorMap tm_r2,
                const __grid_constant__ CUtensorMap tm_c1, const __grid_constant__ CUtensorMap tm_c2,
                __nv_bfloat16* __restrict__ out1, __nv_bfloat16* __restrict__ out2,
                const int* __restrict__ lengths, int* __restrict__ ws, int H, int L) {
   using C = BwdCfg<D, KV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ BwdBarriers<C::ST> bar;
+  __shared__ BwdBarriers<C::ST1, C::ST2> bar;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = &bar.abort;
+  constexpr int kProducerWarp = C::EPI_WARPS;
+  constexpr int kSWarp = C::EPI_WARPS + 1;
+  constexpr int kDPWarp = C::SPLIT_X ? C::EPI_WARPS + 2 : -1;
+  constexpr int kA1Warp = C::EPI_WARPS + (C::SPLIT_X ? 3 : 2);
+  constexpr int kA2Warp = KV ? kA1Warp + 1 : -1;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.r_full, 1);
-    mbar_init(&bar.r_empty, 1);
-    for (int s = 0; s < C::ST; ++s) { mbar_init(&bar.c_full[s], 1); mbar_init(&bar.c_empty[s], 1); }
-    for (int g = 0; g < 2; ++g) { mbar_init(&bar.s_full[g], 1); mbar_init(&bar.p_full[g], 4); }
-    mbar_init(&bar.acc_full, 1);
-    mbar_init(&bar.acc_empty, 8);
-    mbar_init(&bar.drain, 1);
+    mbar_init(&bar.r_empty, C::SPLIT_X ? 2 : 1);
+    for (int s = 0; s < C::ST1; ++s) {
+      mbar_init(&bar.c1_full[s], 1);
+      mbar_init(&bar.c1_empty[s], 2);  // S issuer and A1 issuer
+    }
+    for (int s = 0; s < C::ST2; ++s) {
+      mbar_init(&bar.c2_full[s], 1);
+      mbar_init(&bar.c2_empty[s], KV ? 2 : 1);  // dP issuer (and A2 issuer)
+    }
+    mbar_init(&bar.xs_full, 1);
+    mbar_init(&bar.xdp_full, 1);
+    mbar_init(&bar.xs_read, C::EPI_WARPS);
+    mbar_init(&bar.xdp_read, C::EPI_WARPS);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&bar.p_full[q], 4);
+      mbar_init(&bar.ds_full[q], 4);
+    }
+    mbar_init(&bar.p_free, 1);
+    mbar_init(&bar.ds_free, 1);
+    mbar_init(&bar.acc_full, KV ? 2 : 1);
+    mbar_init(&bar.acc_empty, C::EPI_WARPS);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar.drain[i], 1);
     bar.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kSWarp) {
     tmem_alloc(&bar.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -116,16 +145,32 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = bar.tmem_base;
   const int count = ws[kHdrCount];
 
-  if (warp == 8) {
+  // Descriptor bases (built once, advanced by adding (bytes >> 4): the
+  // start-address field is the low 14 bits and smem stays below 256 KB).
+  const uint32_t sbase = smem_u32(smem);
+  constexpr uint64_t kTile = C::TILE_BYTES >> 4;
+  constexpr uint32_t idesc_x = idesc_bf16_f32(128, C::BN, false, false);
+
+  // X = R C^T over K = D (D/16 steps of K = 16), both operands K-major.
+  auto issue_x = [&](uint32_t d_tmem, uint64_t a0, uint64_t b0) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t off = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+      mma_ss(d_tmem, a0 + off, b0 + off, idesc_x, kk > 0 ? 1u : 0u);
+    }
+  };
+
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_r1);
       tma_prefetch_desc(&tm_r2);
       tma_prefetch_desc(&tm_c1);
       tma_prefetch_desc(&tm_c2);
-      uint32_t st = 0, cph = 0, rph = 0;
-      int c_last[C::ST], r_last = -1;
-      for (int s = 0; s < C::ST; ++s) c_last[s] = -1;
+      uint32_t s1 = 0, p1 = 0, s2 = 0, p2 = 0, rph = 0;
+      int c1_last[C::ST1], c2_last[C::ST2], r_last = -1;
+      for (int s = 0; s < C::ST1; ++s) c1_last[s] = -1;
+      for (int s = 0; s < C::ST2; ++s) c2_last[s] = -1;
       bool ok = true;
       for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
         const Item item = load_item(ws, it);
@@ -140,126 +185,152 @@ __global__ void __launch_bounds__(320, 1)
         r_last = static_cast<int>(rph);
         rph ^= 1;
         for (int j = 0; j < nb; ++j) {
-          if (!(ok = mbar_wait(&bar.c_empty[st], cph ^ 1, abort_flag, ws, 202))) break;
-          mbar_arrive_expect_tx(&bar.c_full[st], 2 * C::TILE_BYTES);
-          uint8_t* c1 = smem + C::OFF_C + st * 2 * C::TILE_BYTES;
-          uint8_t* c2 = c1 + C::TILE_BYTES;
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d(c1 + c * C::BOX_BYTES, &tm_c1, &bar.c_full[st], c * 64, j * C::BN, item.bh);
-            tma_load_3d(c2 + c * C::BOX_BYTES, &tm_c2, &bar.c_full[st], c * 64, j * C::BN, item.bh);
-          }
-          c_last[st] = static_cast<int>(cph);
-          if (++st == C::ST) { st = 0; cph ^= 1; }
+          if (!(ok = mbar_wait(&bar.c1_empty[s1], p1 ^ 1, abort_flag, ws, 202))) break;
+          mbar_arrive_expect_tx(&bar.c1_full[s1], C::TILE_BYTES);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + C::OFF_C1 + s1 * C::TILE_BYTES + c * C::BOX_BYTES, &tm_c1, &bar.c1_full[s1], c * 64,
+                        j * C::BN, item.bh);
+          c1_last[s1] = static_cast<int>(p1);
+          if (++s1 == C::ST1) { s1 = 0; p1 ^= 1; }
+          if (!(ok = mbar_wait(&bar.c2_empty[s2], p2 ^ 1, abort_flag, ws, 203))) break;
+          mbar_arrive_expect_tx(&bar.c2_full[s2], C::TILE_BYTES);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + C::OFF_C2 + s2 * C::TILE_BYTES + c * C::BOX_BYTES, &tm_c2, &bar.c2_full[s2], c * 64,
+                        j * C::BN, item.bh);
+          c2_last[s2] = static_cast<int>(p2);
+          if (++s2 == C::ST2) { s2 = 0; p2 ^= 1; }
         }
       }
       if (!ok) {  // aborting: let the copies in flight land before the CTA exits
         int never = 0;
         volatile int* no_abort = &never;
-        for (int s = 0; s < C::ST; ++s)
-          if (c_last[s] >= 0) mbar_wait(&bar.c_full[s], c_last[s], no_abort, nullptr, 0);
+        for (int s = 0; s < C::ST1; ++s)
+          if (c1_last[s] >= 0) mbar_wait(&bar.c1_full[s], c1_last[s], no_abort, nullptr, 0);
+        for (int s = 0; s < C::ST2; ++s)
+          if (c2_last[s] >= 0) mbar_wait(&bar.c2_full[s], c2_last[s], no_abort, nullptr, 0);
         if (r_last >= 0) mbar_wait(&bar.r_full, r_last, no_abort, nullptr, 0);
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == kSWarp || warp == kDPWarp) {
+    // ------------------------- issuers of S (and, with one region, dP) into X
     if (lane == 0) {
-      constexpr uint32_t idesc_sd = idesc_bf16_f32(128, 64, false, false);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
-      const uint32_t base = smem_u32(smem);
-      uint32_t st = 0, cph = 0, rph = 0, aph = 0;
-      uint32_t pph[2] = {0, 0};
+      const bool is_dp = (warp == kDPWarp);  // separate dP issuer (SPLIT_X only)
+      const uint64_t d_r1 = smem_desc_sw128(sbase + C::OFF_R1, 16, 1024);
+      const uint64_t d_r2 = smem_desc_sw128(sbase + C::OFF_R2, 16, 1024);
+      const uint64_t d_c1 = smem_desc_sw128(sbase + C::OFF_C1, 16, 1024);
+      const uint64_t d_c2 = smem_desc_sw128(sbase + C::OFF_C2, 16, 1024);
+      uint32_t s1 = 0, p1 = 0, s2 = 0, p2 = 0, rph = 0, s_read_ph = 0, dp_read_ph = 0;
       bool ok = true;
-
-      // S_g = R1 C1[g]^T and dP_g = R2 C2[g]^T for the 64 columns of half g.
-      auto issue_sdp = [&](int g, uint32_t s) {
-        const uint32_t c1 = base + C::OFF_C + s * 2 * C::TILE_BYTES + g * 64 * 128;
-        const uint32_t c2 = c1 + C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_S + g * 64, smem_desc_sw128(base + C::OFF_R1 + off, 16, 1024),
-                 smem_desc_sw128(c1 + off, 16, 1024), idesc_sd, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_DP + g * 64, smem_desc_sw128(base + C::OFF_R2 + off, 16, 1024),
-                 smem_desc_sw128(c2 + off, 16, 1024), idesc_sd, kk > 0 ? 1u : 0u);
-        }
-      };
-      // A1 += dS_g C1[g] (and A2 += P_g C2[g]); K = the 64 columns of half g.
-      auto issue_acc = [&](int g, uint32_t s, bool acc) {
-        const uint32_t c1 = base + C::OFF_C + s * 2 * C::TILE_BYTES + g * 64 * 128;
-        const uint32_t c2 = c1 + C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_ts(tmem + C::TM_A1, tmem + C::TM_DP + g * 64 + kk * 8,
-                 smem_desc_sw128(c1 + kk * 2048, C::BOX_BYTES, 1024), idesc_acc, (acc || kk > 0) ? 1u : 0u);
-          if (KV)
-            mma_ts(tmem + C::TM_A2, tmem + C::TM_S + g * 64 + kk * 8,
-                   smem_desc_sw128(c2 + kk * 2048, C::BOX_BYTES, 1024), idesc_acc, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-
       for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
         const Item item = load_item(ws, it);
         const int n = load_len(lengths, item.bh / H, L);
         const int nb = ceil_div(n, C::BN);
         if (!(ok = mbar_wait(&bar.r_full, rph, abort_flag, ws, 211))) break;
         rph ^= 1;
-        if (!(ok = mbar_wait(&bar.c_full[st], cph, abort_flag, ws, 212))) break;
-        tc_fence_after();
-        for (int g = 0; g < 2; ++g) {
-          issue_sdp(g, st);
-          mma_commit(&bar.s_full[g]);
+        for (int j = 0; j < nb; ++j) {
+          if (!is_dp) {
+            // S(j): its region is free once the epilogue has copied out
+            // S(j-1) (separate regions) or dP(j-1) (one shared region).
+            if (!(ok = mbar_wait(&bar.c1_full[s1], p1, abort_flag, ws, 212))) break;
+            if (C::SPLIT_X) {
+              if (!(ok = mbar_wait(&bar.xs_read, s_read_ph ^ 1, abort_flag, ws, 213))) break;
+              s_read_ph ^= 1;
+            } else {
+              if (!(ok = mbar_wait(&bar.xdp_read, dp_read_ph ^ 1, abort_flag, ws, 213))) break;
+              dp_read_ph ^= 1;
+            }
+            tc_fence_after();
+            issue_x(tmem + C::TM_XS, d_r1, d_c1 + s1 * kTile);
+            mma_commit(&bar.xs_full);
+            mma_commit(&bar.c1_empty[s1]);
+            if (++s1 == C::ST1) { s1 = 0; p1 ^= 1; }
+          }
+          if (is_dp || !C::SPLIT_X) {
+            // dP(j): free once dP(j-1) (separate regions) or S(j) (one shared
+            // region) has been copied out.
+            if (!(ok = mbar_wait(&bar.c2_full[s2], p2, abort_flag, ws, 214))) break;
+            if (C::SPLIT_X) {
+              if (!(ok = mbar_wait(&bar.xdp_read, dp_read_ph ^ 1, abort_flag, ws, 215))) break;
+              dp_read_ph ^= 1;
+            } else {
+              if (!(ok = mbar_wait(&bar.xs_read, s_read_ph, abort_flag, ws, 215))) break;
+              s_read_ph ^= 1;
+            }
+            tc_fence_after();
+            issue_x(tmem + C::TM_XDP, d_r2, d_c2 + s2 * kTile);
+            mma_commit(&bar.xdp_full);
+            mma_commit(&bar.c2_empty[s2]);
+            if (++s2 == C::ST2) { s2 = 0; p2 ^= 1; }
+          }
+          if (j + 1 == nb) mma_commit(&bar.r_empty);
         }
-        if (nb == 1) mma_commit(&bar.r_empty);
+      }
+      int never = 0;
+      mma_commit(&bar.drain[is_dp ? 1 : 0]);
+      mbar_wait(&bar.drain[is_dp ? 1 : 0], 0, &never, ws, 219);
+    }
+  } else if (warp == kA1Warp || warp == kA2Warp) {
+    // -------------------------- issuers of A1 += dS C1 and (dK/dV) A2 += P C2
+    if (lane == 0) {
+      const bool second = (warp == kA2Warp);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+      // MN-major view of the C1 (A1) or C2 (A2) ring: rows = the K dimension.
+      const uint64_t d_cmn = smem_desc_sw128(sbase + (second ? C::OFF_C2 : C::OFF_C1), C::BOX_BYTES, 1024);
+      const int slots = second ? C::ST2 : C::ST1;
+      uint64_t* cfull = second ? bar.c2_full : bar.c1_full;
+      uint64_t* cempty = second ? bar.c2_empty : bar.c1_empty;
+      const uint32_t tm_acc = tmem + (second ? C::TM_A2 : C::TM_A1);
+      const uint32_t tm_a = tmem + (second ? C::TM_P : C::TM_DS);
+      uint64_t* full = second ? bar.p_full : bar.ds_full;
+      uint64_t* freed = second ? &bar.p_free : &bar.ds_free;
+      uint32_t st = 0, cph = 0, aph = 0;
+      uint32_t fph[4] = {0, 0, 0, 0};
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
+        const Item item = load_item(ws, it);
+        const int n = load_len(lengths, item.bh / H, L);
+        const int nb = ceil_div(n, C::BN);
         for (int j = 0; ok && j < nb; ++j) {
-          const bool has_next = (j + 1 < nb);
-          const uint32_t cur = st;
-          uint32_t nxt = st + 1, nph = cph;
-          if (nxt == C::ST) { nxt = 0; nph ^= 1; }
-          for (int g = 0; g < 2; ++g) {
-            if (!(ok = mbar_wait(&bar.p_full[g], pph[g], abort_flag, ws, 213))) break;
-            pph[g] ^= 1;
-            if (j == 0 && g == 0) {
-              if (!(ok = mbar_wait(&bar.acc_empty, aph ^ 1, abort_flag, ws, 214))) break;
+          if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 231))) break;
+          const uint64_t b0 = d_cmn + st * kTile;
+          for (int q = 0; q < 4; ++q) {
+            if (!(ok = mbar_wait(&full[q], fph[q], abort_flag, ws, 232))) break;
+            fph[q] ^= 1;
+            const bool first = (j == 0 && q == 0);
+            if (first) {
+              if (!(ok = mbar_wait(&bar.acc_empty, aph ^ 1, abort_flag, ws, 233))) break;
               aph ^= 1;
             }
             tc_fence_after();
-            issue_acc(g, cur, !(j == 0 && g == 0));
-            if (has_next) {
-              if (g == 0) {
-                if (!(ok = mbar_wait(&bar.c_full[nxt], nph, abort_flag, ws, 215))) break;
-                tc_fence_after();
-              }
-              issue_sdp(g, nxt);
-              mma_commit(&bar.s_full[g]);
-            }
+            // K = the chunk's 32 columns: two K=16 steps; the chunk's bf16
+            // values sit in 16 TMEM columns (two per column).
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_ts(tm_acc, tm_a + q * 16 + kk * 8, b0 + ((q * 32 * 128 + kk * 2048) >> 4), idesc_acc,
+                     (first && kk == 0) ? 0u : 1u);
           }
           if (!ok) break;
-          if (has_next && j + 2 == nb) mma_commit(&bar.r_empty);
-          mma_commit(&bar.c_empty[cur]);
-          st = nxt;
-          cph = nph;
+          mma_commit(freed);
+          mma_commit(&cempty[st]);
+          if (++st == slots) { st = 0; cph ^= 1; }
         }
         if (!ok) break;
         mma_commit(&bar.acc_full);
       }
       int never = 0;
-      mma_commit(&bar.drain);
-      mbar_wait(&bar.drain, 0, &never, ws, 219);
+      mma_commit(&bar.drain[second ? 3 : 2]);
+      mbar_wait(&bar.drain[second ? 3 : 2], 0, &never, ws, 239);
     }
-  } else {
+  } else if (warp < C::EPI_WARPS) {
     // ------------------------------------------------------------- epilogue
-    const int g = warp >> 2;                      // column half of this warpgroup
+    const int g = warp >> 2;                      // column half: chunks 2g, 2g+1
     const int r = ((warp & 3) << 5) + lane;       // row within the item = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
-    const uint32_t tS = tmem + lane_off + C::TM_S + g * 64;
-    const uint32_t tDP = tmem + lane_off + C::TM_DP + g * 64;
+    const uint32_t tXS = tmem + lane_off + C::TM_XS + g * 64;
+    const uint32_t tXDP = tmem + lane_off + C::TM_XDP + g * 64;
     constexpr float scale = Scale<D>::value;
     constexpr float half_scale = 0.5f * scale;
-    uint32_t sph = 0, aph = 0;
+    uint32_t s_ph = 0, dp_ph = 0, free_ph = 0, aph = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
       const Item item = load_item(ws, it);
@@ -267,83 +338,138 @@ __global__ void __launch_bounds__(320, 1)
       const int nb = ceil_div(n, C::BN);
       const float half_bias = -0.5f * __logf(static_cast<float>(n));
       for (int j = 0; j < nb; ++j) {
-        if (!(ok = mbar_wait(&bar.s_full[g], sph, abort_flag, ws, 221))) break;
-        sph ^= 1;
+        // ---- S -> P (fp32 kept in registers for dS), bf16 P for dV
+        float p[64];
+        uint32_t dp[2][32];
+        {
+          uint32_t s0[32], s1[32];
+          if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, ws, 221))) break;
+          s_ph ^= 1;
+          tc_fence_after();
+          tmem_ld32x2(tXS, tXS + 32, s0, s1);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.xs_read);
+          if (!C::SPLIT_X) {
+            // One shared region: copy dP out as soon as it lands, so that the
+            // next block's S can be computed while this epilogue works.
+            if (!(ok = mbar_wait(&bar.xdp_full, dp_ph, abort_flag, ws, 222))) break;
+            dp_ph ^= 1;
+            tc_fence_after();
+            tmem_ld32x2(tXDP, tXDP + 32, dp[0], dp[1]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.xdp_read);
+          }
+          const int valid = n - (j * C::BN + g * 64);  // columns < valid are real tokens
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            p[e] = sigmoid_from_score(__uint_as_float(s0[e]), half_scale, half_bias);
+            p[32 + e] = sigmoid_from_score(__uint_as_float(s1[e]), half_scale, half_bias);
+          }
+          if (valid < 64) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) p[e] = (e < valid) ? p[e] : 0.f;
+          }
+        }
+        if (KV) {
+          if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(p[32 * c + 2 * e], p[32 * c + 2 * e + 1]);
+            tmem_st16(tmem + lane_off + C::TM_P + (2 * g + c) * 16, pk);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.p_full[2 * g + c]);
+          }
+        }
+        // ---- dP -> dS = dP P (1 - P), bf16 dS for dQ / dK
+        if (C::SPLIT_X) {
+          if (!(ok = mbar_wait(&bar.xdp_full, dp_ph, abort_flag, ws, 222))) break;
+          dp_ph ^= 1;
+        }
+        if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, ws, 224))) break;
+        free_ph ^= 1;
         tc_fence_after();
-        const int valid = n - (j * C::BN + g * 64);  // columns < valid are real tokens
+        if (C::SPLIT_X && C::DP_BOTH) {
+          tmem_ld32x2(tXDP, tXDP + 32, dp[0], dp[1]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.xdp_read);
+        }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          uint32_t s[32], dp[32];
-          tmem_ld32x2(tS + c * 32, tDP + c * 32, s, dp);
-          uint32_t pk_p[16], pk_ds[16];
+          if (C::SPLIT_X && !C::DP_BOTH) {
+            tmem_ld32(tXDP + 32 * c, dp[c]);
+            if (c == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bar.xdp_read);
+            }
+          }
+          uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float p0 = sigmoid_from_score(__uint_as_float(s[2 * e]), half_scale, half_bias);
-            float p1 = sigmoid_from_score(__uint_as_float(s[2 * e + 1]), half_scale, half_bias);
-            if (valid < 64) {
-              const int col = c * 32 + 2 * e;
-              p0 = (col < valid) ? p0 : 0.f;
-              p1 = (col + 1 < valid) ? p1 : 0.f;
-            }
-            const float ds0 = __uint_as_float(dp[2 * e]) * (p0 - p0 * p0);
-            const float ds1 = __uint_as_float(dp[2 * e + 1]) * (p1 - p1 * p1);
-            pk_p[e] = pack_bf16x2(p0, p1);
-            pk_ds[e] = pack_bf16x2(ds0, ds1);
+            const float q0 = p[32 * c + 2 * e], q1 = p[32 * c + 2 * e + 1];
+            const float ds0 = __uint_as_float(dp[c][2 * e]) * (q0 - q0 * q0);
+            const float ds1 = __uint_as_float(dp[c][2 * e + 1]) * (q1 - q1 * q1);
+            pk[e] = pack_bf16x2(ds0, ds1);
           }
-          // bf16 results for columns [32c, 32c+32) go to TMEM columns
-          // [16c, 16c+16) of the same region: already read by this thread.
-          if (KV) tmem_st16(tS + c * 16, pk_p);
-          tmem_st16(tDP + c * 16, pk_ds);
+          tmem_st16(tmem + lane_off + C::TM_DS + (2 * g + c) * 16, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.ds_full[2 * g + c]);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar.p_full[g]);
       }
       if (!ok) break;
-      if (!(ok = mbar_wait(&bar.acc_full, aph, abort_flag, ws, 222))) break;
+      if (!(ok = mbar_wait(&bar.acc_full, aph, abort_flag, ws, 225))) break;
       aph ^= 1;
       tc_fence_after();
       const int row = item.blk * C::BM + r;
       const bool in_range = row < L;
       const bool valid_row = row < n;
       const size_t row_off = (static_cast<size_t>(item.bh) * L + row) * D;
-      if (!KV) {
-        // dQ: warpgroup g writes columns [g*D/2, (g+1)*D/2) of A1 * scale.
+      // 32-column chunks of the accumulators: A1 (-> out1, times scale), then
+      // A2 (-> out2) for dK/dV; each half of the warps takes every other
+      // chunk. All of a thread's chunks are copied out first, so the
+      // accumulators are released before the (slower) global stores.
+      constexpr int kChunks = (KV ? 2 : 1) * (D / 32);
+      constexpr int kPer = kChunks / 2;
+      uint32_t v[kPer][32];
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          const int col = g * (D / 2) + c * 32;
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + C::TM_A1 + col, v);
-          if (in_range) {
-            if (valid_row) store_row32(out1 + row_off + col, v, scale);
-            else store_zero32(out1 + row_off + col);
-          }
-        }
-      } else {
-        // dK (= A1 * scale) by warpgroup 0, dV (= A2) by warpgroup 1.
-        const uint32_t tA = tmem + lane_off + (g == 0 ? C::TM_A1 : C::TM_A2);
-        __nv_bfloat16* dst = (g == 0 ? out1 : out2) + row_off;
-        const float mul = (g == 0) ? scale : 1.0f;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tA + c * 32, v);
-          if (in_range) {
-            if (valid_row) store_row32(dst + c * 32, v, mul);
-            else store_zero32(dst + c * 32);
-          }
-        }
+      for (int i = 0; i < kPer; ++i) {
+        const int c = g + 2 * i;
+        const bool second = c >= D / 32;
+        const int col = (second ? c - D / 32 : c) * 32;
+        tmem_ld32_async(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v[i]);
       }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) tmem_ld_wait32(v[i]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.acc_empty);
+      if (in_range) {
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+          const int c = g + 2 * i;
+          const bool second = c >= D / 32;
+          const int col = (second ? c - D / 32 : c) * 32;
+          __nv_bfloat16* dst = (second ? out2 : out1) + row_off + col;
+          if (valid_row) store_row32(dst, v[i], second ? 1.0f : scale);
+          else store_zero32(dst);
+        }
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kSWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

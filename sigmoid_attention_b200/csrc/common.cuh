@@ -66,12 +66,22 @@ __device__ __forceinline__ float sigmoid_from_score(float s, float half_scale, f
   return fmaf(t, 0.5f, 0.5f);
 }
 
-// Store `D` bf16 zeros at `dst` (16-byte aligned, D a multiple of 8).
-template <int D>
-__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst) {
+// Convert 32 fp32 accumulator values (times `mul`) to bf16 and store them.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul) {
   uint4* p = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int i = 0; i < D / 8; ++i) p[i] = make_uint4(0, 0, 0, 0);
+  for (int q = 0; q < 4; ++q) {
+    p[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q + 0]) * mul, __uint_as_float(v[8 * q + 1]) * mul),
+                      pack_bf16x2(__uint_as_float(v[8 * q + 2]) * mul, __uint_as_float(v[8 * q + 3]) * mul),
+                      pack_bf16x2(__uint_as_float(v[8 * q + 4]) * mul, __uint_as_float(v[8 * q + 5]) * mul),
+                      pack_bf16x2(__uint_as_float(v[8 * q + 6]) * mul, __uint_as_float(v[8 * q + 7]) * mul));
+  }
+}
+
+__device__ __forceinline__ void store_zero32(__nv_bfloat16* dst) {
+  uint4* p = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) p[q] = make_uint4(0, 0, 0, 0);
 }
 
 }  // namespace sigattn

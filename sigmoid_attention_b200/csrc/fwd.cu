@@ -7,19 +7,27 @@
 // rescale: sec. 2A "decoupling"), so one pass over the key blocks suffices and
 // the accumulator is never rescaled.
 //
-// Design (one persistent CTA per SM, 320 threads):
-//   warps 0-3  epilogue for query tile 0 (TMEM lanes 0..127 = its 128 rows)
-//   warps 4-7  epilogue for query tile 1
-//   warp  8    TMA producer: Q tiles once per item, then a ring of K and V tiles
-//   warp  9    TMEM allocator and the single thread that issues tcgen05.mma
+// Design (one persistent CTA per SM, 608 threads):
+//   warps 0-7   epilogue for query tile 0 (TMEM lanes 0..127 = its 128 rows):
+//               warps 0-3 key columns 0-63, warps 4-7 key columns 64-127
+//   warps 8-15  epilogue for query tile 1, split the same way
+//   warp  16    TMA producer: Q tiles once per item, then a ring of K and V tiles
+//   warps 17,18 one tcgen05.mma issuer per query tile (warp 17 also owns TMEM).
+// A single thread issues a tcgen05.mma only every ~100 cycles, which is more
+// than a 128x128x16 product takes, so each tile has its own issuing thread;
+// each issuer keeps its tile's products in order (S_t(j+1) overwrites P_t(j)
+// only after PV_t(j) was issued by the same thread).
 // A work item is 256 query rows (two 128-row tiles) of one (b, h); both tiles
 // share every K/V block that is loaded. Per key block j and tile t:
 //   S_t = Q_t K_j^T          tcgen05.mma, A and B from shared memory, fp32 in TMEM
 //   P_t = sigma(S_t*scale+b) epilogue warps: TMEM -> registers -> bf16 P back
-//                            into the first 64 columns of S_t's TMEM region
+//                            over the first 32 columns of each 64-column half
 //   O_t += P_t V_j           tcgen05.mma with A = P_t read from TMEM
-// The MMA issue order S0(j), S1(j), PV0(j), S0(j+1), PV1(j), S1(j+1), ... lets
-// one tile's epilogue run while the tensor core works on the other tile.
+// Per tile the issue order is S_t(j), PV_t(j) (after P_t(j)), S_t(j+1), ...
+// The two tiles' epilogues take turns (tile 1's sigmoid pass over block j
+// starts when tile 0's is done, tile 0's pass over j+1 when tile 1's j is
+// done): each has the MUFU pipe to itself while the tensor core works on the
+// other tile, instead of both tiles running in phase.
 // TMEM: S/P of tile t at columns [128t, 128t+128), O of tile t at 256 + t*D.
 #include "common.cuh"
 
@@ -42,7 +50,8 @@ struct FwdCfg {
   static constexpr int TM_S = 0;
   static constexpr int TM_O = 256;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static constexpr int EPI_WARPS = 16;
+  static constexpr int THREADS = (EPI_WARPS + 3) * 32;
 };
 
 template <int KST, int VST>
@@ -50,14 +59,15 @@ struct FwdBarriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
-  uint64_t drain;
+  uint64_t s_full[2], p_full[4], o_full[2], o_empty[2];
+  uint64_t epi_done[2];  // tile t's warps finished their sigmoid pass over a block
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__((16 + 3) * 32, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                const int* __restrict__ lengths, int* __restrict__ ws, int H, int L) {
@@ -74,21 +84,27 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = &bar.abort;
 
   if (threadIdx.x == 0) {
+    // "empty" barriers take one arrival from each of the two issuers
     mbar_init(&bar.q_full, 1);
-    mbar_init(&bar.q_empty, 1);
-    for (int s = 0; s < C::KST; ++s) { mbar_init(&bar.k_full[s], 1); mbar_init(&bar.k_empty[s], 1); }
-    for (int s = 0; s < C::VST; ++s) { mbar_init(&bar.v_full[s], 1); mbar_init(&bar.v_empty[s], 1); }
+    mbar_init(&bar.q_empty, 2);
+    for (int s = 0; s < C::KST; ++s) { mbar_init(&bar.k_full[s], 1); mbar_init(&bar.k_empty[s], 2); }
+    for (int s = 0; s < C::VST; ++s) { mbar_init(&bar.v_full[s], 1); mbar_init(&bar.v_empty[s], 2); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar.s_full[t], 1);
-      mbar_init(&bar.p_full[t], 4);
+      mbar_init(&bar.p_full[2 * t], 4);
+      mbar_init(&bar.p_full[2 * t + 1], 4);
       mbar_init(&bar.o_full[t], 1);
-      mbar_init(&bar.o_empty[t], 4);
+      mbar_init(&bar.o_empty[t], 8);
     }
-    mbar_init(&bar.drain, 1);
+    mbar_init(&bar.epi_done[0], 8);
+    mbar_init(&bar.epi_done[1], 8);
+    mbar_init(&bar.drain[0], 1);
+    mbar_init(&bar.drain[1], 1);
     bar.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  constexpr int kProducerWarp = C::EPI_WARPS, kMmaWarp = C::EPI_WARPS + 1;  // issuers: kMmaWarp + t
+  if (warp == kMmaWarp) {
     tmem_alloc(&bar.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -98,7 +114,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = bar.tmem_base;
   const int count = ws[kHdrCount];
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -152,35 +168,43 @@ __global__ void __launch_bounds__(320, 1)
         if (q_last >= 0) mbar_wait(&bar.q_full, q_last, no_abort, nullptr, 0);
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= kMmaWarp) {
+    // ------------------------------------------------------- MMA issuer of tile t
+    const int t = warp - kMmaWarp;
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, C::BN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       uint32_t kst = 0, kph = 0, vst = 0, vph = 0, qph = 0;
-      uint32_t pph[2] = {0, 0}, oph[2] = {0, 0};
+      uint32_t pph[2] = {0, 0}, oph = 0;
       bool ok = true;
+      // Descriptors are built once and advanced by adding (bytes >> 4): the
+      // start-address field is the low 14 bits and smem stays below 256 KB.
+      const uint64_t d_q = smem_desc_sw128(q_addr, 16, 1024) + ((t * C::TILE_BYTES) >> 4);
+      const uint64_t d_k = smem_desc_sw128(k_addr, 16, 1024);
+      const uint64_t d_v = smem_desc_sw128(v_addr, C::BOX_BYTES, 1024);  // MN-major view of V
+      constexpr uint64_t kTile = C::TILE_BYTES >> 4;
+      const uint32_t tm_s = tmem + C::TM_S + t * 128;
+      const uint32_t tm_o = tmem + C::TM_O + t * D;
 
-      auto issue_s = [&](int t, uint32_t ks) {
-        const uint32_t d_tmem = tmem + C::TM_S + t * 128;
+      auto issue_s = [&](uint32_t ks) {
+        const uint64_t b0 = d_k + ks * kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(q_addr + t * C::TILE_BYTES + off, 16, 1024);
-          const uint64_t b = smem_desc_sw128(k_addr + ks * C::TILE_BYTES + off, 16, 1024);
-          mma_ss(d_tmem, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t off = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+          mma_ss(tm_s, d_q + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, uint32_t vs, bool acc) {
-        const uint32_t d_tmem = tmem + C::TM_O + t * D;
-        const uint32_t a_tmem = tmem + C::TM_S + t * 128;
+      // O_t += P_t[:, 64h : 64h+64] V_j[64h : 64h+64, :] for key half h: P of
+      // that half sits in TMEM columns [128t + 64h, 128t + 64h + 32).
+      auto issue_pv = [&](int h, uint32_t vs, bool acc) {
+        const uint64_t b0 = d_v + vs * kTile + ((h * 64 * 128) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint64_t b = smem_desc_sw128(v_addr + vs * C::TILE_BYTES + kk * 2048, C::BOX_BYTES, 1024);
-          mma_ts(d_tmem, a_tmem + kk * 8, b, idesc_o, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tm_o, tm_s + h * 64 + kk * 8, b0 + ((kk * 2048) >> 4), idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
+      auto advance_k = [&]() { if (++kst == C::KST) { kst = 0; kph ^= 1; } };
+      auto advance_v = [&]() { if (++vst == C::VST) { vst = 0; vph ^= 1; } };
 
       for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
         const Item item = load_item(ws, it);
@@ -188,75 +212,90 @@ __global__ void __launch_bounds__(320, 1)
         const int row0 = item.blk * (C::BM * C::NQ);
         const int ntiles = (row0 + C::BM < n) ? 2 : 1;
         const int nkb = ceil_div(n, C::BN);
+        if (t >= ntiles) {
+          // Tile 1 is fully padded in this item. Its issuer issues nothing but
+          // still waits for every load and gives its arrival on every shared
+          // "empty" barrier, so both issuers stay in step with the rings.
+          if (!(ok = mbar_wait(&bar.q_full, qph, abort_flag, ws, 117))) break;
+          qph ^= 1;
+          for (int j = 0; ok && j < nkb; ++j) {
+            if (!(ok = mbar_wait(&bar.k_full[kst], kph, abort_flag, ws, 117))) break;
+            mma_commit(&bar.k_empty[kst]);
+            advance_k();
+            if (!(ok = mbar_wait(&bar.v_full[vst], vph, abort_flag, ws, 117))) break;
+            mma_commit(&bar.v_empty[vst]);
+            advance_v();
+          }
+          mma_commit(&bar.q_empty);
+          continue;
+        }
         if (!(ok = mbar_wait(&bar.q_full, qph, abort_flag, ws, 111))) break;
         qph ^= 1;
         if (!(ok = mbar_wait(&bar.k_full[kst], kph, abort_flag, ws, 112))) break;
         tc_fence_after();
-        for (int t = 0; t < ntiles; ++t) {
-          issue_s(t, kst);
-          mma_commit(&bar.s_full[t]);
-        }
+        issue_s(kst);
+        mma_commit(&bar.s_full[t]);
         if (nkb == 1) mma_commit(&bar.q_empty);
         mma_commit(&bar.k_empty[kst]);
-        if (++kst == C::KST) { kst = 0; kph ^= 1; }
+        advance_k();
 
         for (int j = 0; ok && j < nkb; ++j) {
           const bool has_next = (j + 1 < nkb);
           if (!(ok = mbar_wait(&bar.v_full[vst], vph, abort_flag, ws, 113))) break;
-          tc_fence_after();
-          for (int t = 0; t < ntiles; ++t) {
-            if (!(ok = mbar_wait(&bar.p_full[t], pph[t], abort_flag, ws, 114))) break;
-            pph[t] ^= 1;
-            if (j == 0) {
-              if (!(ok = mbar_wait(&bar.o_empty[t], oph[t] ^ 1, abort_flag, ws, 115))) break;
-              oph[t] ^= 1;
+          for (int h = 0; h < 2; ++h) {
+            if (!(ok = mbar_wait(&bar.p_full[2 * t + h], pph[h], abort_flag, ws, 114))) break;
+            pph[h] ^= 1;
+            if (j == 0 && h == 0) {
+              if (!(ok = mbar_wait(&bar.o_empty[t], oph ^ 1, abort_flag, ws, 115))) break;
+              oph ^= 1;
             }
             tc_fence_after();
-            issue_pv(t, vst, j > 0);
-            if (has_next) {
-              if (t == 0) {
-                if (!(ok = mbar_wait(&bar.k_full[kst], kph, abort_flag, ws, 116))) break;
-                tc_fence_after();
-              }
-              issue_s(t, kst);
-              mma_commit(&bar.s_full[t]);
-            }
+            issue_pv(h, vst, j > 0 || h > 0);
           }
           if (!ok) break;
+          mma_commit(&bar.v_empty[vst]);
+          advance_v();
           if (has_next) {
+            if (!(ok = mbar_wait(&bar.k_full[kst], kph, abort_flag, ws, 116))) break;
+            tc_fence_after();
+            issue_s(kst);
+            mma_commit(&bar.s_full[t]);
             if (j + 2 == nkb) mma_commit(&bar.q_empty);
             mma_commit(&bar.k_empty[kst]);
-            if (++kst == C::KST) { kst = 0; kph ^= 1; }
+            advance_k();
           }
-          mma_commit(&bar.v_empty[vst]);
-          if (++vst == C::VST) { vst = 0; vph ^= 1; }
         }
         if (!ok) break;
-        for (int t = 0; t < ntiles; ++t) mma_commit(&bar.o_full[t]);
+        mma_commit(&bar.o_full[t]);
       }
       // Wait for every MMA issued so far before TMEM can be released.
       int never = 0;
-      mma_commit(&bar.drain);
-      mbar_wait(&bar.drain, 0, &never, ws, 119);
+      mma_commit(&bar.drain[t]);
+      mbar_wait(&bar.drain[t], 0, &never, ws, 119);
     }
   } else {
     // ------------------------------------------------------------- epilogue
-    const int t = warp >> 2;                       // query tile of this warpgroup
+    const int t = warp >> 3;                       // query tile of this warp
+    const int h = (warp >> 2) & 1;                 // key half (64 columns) of this warp
     const int r = ((warp & 3) << 5) + lane;        // row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
-    const uint32_t tS = tmem + lane_off + C::TM_S + t * 128;
-    const uint32_t tO = tmem + lane_off + C::TM_O + t * D;
+    const uint32_t tS = tmem + lane_off + C::TM_S + t * 128 + h * 64;
+    const uint32_t tO = tmem + lane_off + C::TM_O + t * D + h * (D / 2);
     constexpr float half_scale = 0.5f * Scale<D>::value;
-    uint32_t sph = 0, oph = 0;
+    uint32_t sph = 0, oph = 0, turn_ph = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
       const Item item = load_item(ws, it);
       const int n = load_len(lengths, item.bh / H, L);
+      const bool two_tiles = item.blk * (C::BM * C::NQ) + C::BM < n;
       const int row0 = item.blk * (C::BM * C::NQ) + t * C::BM;
       const int row = row0 + r;
-      __nv_bfloat16* orow = out + (static_cast<size_t>(item.bh) * L + row) * D;
+      __nv_bfloat16* orow = out + (static_cast<size_t>(item.bh) * L + row) * D + h * (D / 2);
       if (row0 >= n) {  // tile fully padded: its rows of O are zero
-        if (row < L) store_zero_row<D>(orow);
+        if (row < L) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) store_zero32(orow + c * 32);
+        }
         continue;
       }
       const int nkb = ceil_div(n, C::BN);
@@ -264,72 +303,70 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; j < nkb; ++j) {
         if (!(ok = mbar_wait(&bar.s_full[t], sph, abort_flag, ws, 121))) break;
         sph ^= 1;
+        // Take turns with the other tile (two-tile items only): tile 1 waits
+        // for tile 0's pass over block j, tile 0 for tile 1's pass over j-1.
+        if (two_tiles && (t == 1 || j > 0)) {
+          if (!(ok = mbar_wait(&bar.epi_done[1 - t], turn_ph, abort_flag, ws, 123))) break;
+          turn_ph ^= 1;
+        }
         tc_fence_after();
-        const int valid = n - j * C::BN;  // columns < valid are real keys
+        const int valid = n - (j * C::BN + h * 64);  // columns < valid are real keys
+        // The half's 64 keys in two 32-column chunks; P of chunk c goes to
+        // TMEM columns [16c, 16c + 16) of the half, which hold S values this
+        // thread has already read (chunk 0's).
 #pragma unroll
-        for (int c = 0; c < 4; c += 2) {
-          uint32_t a[32], b[32];
-          tmem_ld32x2(tS + c * 32, tS + (c + 1) * 32, a, b);
-          uint32_t pa[16], pb[16];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tS + 32 * c, a);
+          uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             float p0 = sigmoid_from_score(__uint_as_float(a[2 * e]), half_scale, half_bias);
             float p1 = sigmoid_from_score(__uint_as_float(a[2 * e + 1]), half_scale, half_bias);
-            float p2 = sigmoid_from_score(__uint_as_float(b[2 * e]), half_scale, half_bias);
-            float p3 = sigmoid_from_score(__uint_as_float(b[2 * e + 1]), half_scale, half_bias);
-            if (valid < C::BN) {
-              const int col = c * 32 + 2 * e;
-              p0 = (col < valid) ? p0 : 0.f;
-              p1 = (col + 1 < valid) ? p1 : 0.f;
-              p2 = (col + 32 < valid) ? p2 : 0.f;
-              p3 = (col + 33 < valid) ? p3 : 0.f;
+            if (valid < 64) {
+              p0 = (32 * c + 2 * e < valid) ? p0 : 0.f;
+              p1 = (32 * c + 2 * e + 1 < valid) ? p1 : 0.f;
             }
-            pa[e] = pack_bf16x2(p0, p1);
-            pb[e] = pack_bf16x2(p2, p3);
+            pk[e] = pack_bf16x2(p0, p1);
           }
-          // P for columns [32c, 32c+64) goes to TMEM columns [16c, 16c+32),
-          // which only overlap S columns this thread has already read.
-          tmem_st16(tS + c * 16, pa);
-          tmem_st16(tS + c * 16 + 16, pb);
+          tmem_st16(tS + 16 * c, pk);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar.p_full[t]);
+        if (lane == 0) {
+          mbar_arrive(&bar.p_full[2 * t + h]);
+          // Hand the turn over: every pass of tile 0 is awaited by tile 1;
+          // tile 1's last pass of the item has no successor to wait for it.
+          if (two_tiles && (t == 0 || j + 1 < nkb)) mbar_arrive(&bar.epi_done[t]);
+        }
       }
       if (!ok) break;
       if (!(ok = mbar_wait(&bar.o_full[t], oph, abort_flag, ws, 122))) break;
       oph ^= 1;
       tc_fence_after();
+      // This warp's D/2 columns of O: copy them all out, release O, then store.
+      uint32_t v[D / 64][32];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tO + c * 32, v);
-        if (row < L) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-          if (row < n) {
+      for (int c = 0; c < D / 64; ++c) tmem_ld32_async(tO + c * 32, v[c]);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1])),
-                                  pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                                  pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                                  pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
-          }
-        }
-      }
+      for (int c = 0; c < D / 64; ++c) tmem_ld_wait32(v[c]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.o_empty[t]);
+      if (row < L) {
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          if (row < n) store_row32(orow + c * 32, v[c], 1.0f);
+          else store_zero32(orow + c * 32);
+        }
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
