@@ -78,14 +78,14 @@ bool device_info(DeviceInfo* out) {
 }
 
 // 3-D view {d, Lmax, B*H} of a [B][H][Lmax][d] bf16 tensor, loaded as
-// [128 rows][64 columns] boxes with the 128-byte swizzle the tcgen05
+// [box_rows rows][64 columns] boxes with the 128-byte swizzle the tcgen05
 // descriptors expect. Rows past Lmax read as zeros.
-bool make_map(CUtensorMap* map, const void* ptr, int BH, int L, int d) {
+bool make_map(CUtensorMap* map, const void* ptr, int BH, int L, int d, int box_rows = 128) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t elem[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, elem,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -210,9 +210,12 @@ int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* do
   if (st != SIGATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
     return SIGATTN_ERR_INVALID_ARG;
+  // K, V are the row operands (128-row boxes); Q, dO are streamed in blocks of
+  // bwd_col_block(true, d) rows.
+  const int cb = bwd_col_block(true, d);
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) ||
-      !make_map(&tv, v, B * H, Lmax, d) || !make_map(&tdo, dout, B * H, Lmax, d))
+  if (!make_map(&tq, q, B * H, Lmax, d, cb) || !make_map(&tk, k, B * H, Lmax, d) ||
+      !make_map(&tv, v, B * H, Lmax, d) || !make_map(&tdo, dout, B * H, Lmax, d, cb))
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);

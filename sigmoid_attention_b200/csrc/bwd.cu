@@ -18,27 +18,24 @@
 //   dK/dV(KV=1) keys    K  V  |        Q   dO | K Q^T    V dO^T    A1 += dS^T Q    -> dK
 //                                                                   A2 += P^T dO    -> dV
 //
-// Per 128-column block j, in tensor memory (TMEM):
+// Per block j of BN columns, in tensor memory (TMEM):
 //   XS  = R1 C1_j^T  (S,  fp32)  -> epilogue: P = sigma(S*scale + b), 0 for
 //                                   padded columns; bf16 P to its own region
 //   XdP = R2 C2_j^T  (dP, fp32)  -> epilogue: dS = dP P (1 - P); bf16 dS to
 //                                   its own region
 //   A1 += dS C1_j, A2 += P C2_j  (A operand read from TMEM, per 32-column chunk)
 // A region is released as soon as the epilogue has copied it to registers, so
-// the products of block j+1 overlap the epilogue of block j. S comes first:
-// P, and with it the dV products and the release of C2, are ready before dP.
-// One thread issues a tcgen05.mma only every ~100 cycles, so the products are
-// spread over several issuing warps: S, dP (when they have separate TMEM
-// regions), A1 and A2. C1 and C2 have rings of their own: C2 (V for dQ, dO
-// for dK/dV) is released earlier than C1, so C1 gets the deeper ring.
+// the products of block j+1 overlap the epilogue of block j. One thread issues
+// a tcgen05.mma only every ~100 cycles, so the products are spread over four
+// issuing warps (S, dP, A1, A2), each with its own TMEM region. C1 and C2 have
+// rings of their own.
 //
-// TMEM columns (512): with separate S and dP regions (dQ, and dK/dV at D=64):
-//   XS [0,128) XdP [128,256) P [256,320) dS [320,384) A1 [384,384+D) A2 after;
-// dK/dV at D=128 has room for one region X [0,128) that holds S, then dP:
-//   X [0,128) P [128,192) dS [192,256) A1 [256,384) A2 [384,512).
-// Warps: 0-7 epilogue (0-3: columns 0-63, 4-7: columns 64-127), 8 TMA
-// producer, then the issuers: S (owns TMEM), dP (separate regions only), A1,
-// A2 (dK/dV only).
+// BN is 128, except for dK/dV at D = 128, where the two D-wide accumulators
+// leave room in the 512 TMEM columns only for 64-column S and dP regions:
+//   XS [0,BN) XdP [BN,2BN) P [2BN,2.5BN) dS [2.5BN,3BN) A1 [3BN,3BN+D) A2 after.
+// Warps: 0-7 epilogue (warps 4g..4g+3 take columns [g BN/2, (g+1) BN/2) of
+// each block), 8 TMA producer, 9 S issuer (owns TMEM), 10 dP issuer, 11 A1
+// issuer, 12 A2 issuer (dK/dV only).
 #include "common.cuh"
 
 namespace sigattn {
@@ -46,31 +43,33 @@ namespace sigattn {
 template <int D, bool KV>
 struct BwdCfg {
   static constexpr int BM = kBwdItemRows;   // 128 rows per item
-  static constexpr int BN = kColBlock;      // 128 columns per block
-  static constexpr bool SPLIT_X = !(KV && D == 128);
-  static constexpr int ST1 = (D == 128) ? 3 : 4;   // C1 ring slots
-  static constexpr int ST2 = (D == 128) ? 2 : 4;   // C2 ring slots
-  static constexpr int BOX_BYTES = 128 * 64 * 2;
-  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int BN = bwd_col_block(KV, D);
+  static constexpr int NCH = BN / 32;       // 32-column chunks per block
+  static constexpr int CPW = NCH / 2;       // chunks per epilogue warp
+  static constexpr int BOX_R = 128 * 64 * 2;   // [128 rows][64 cols] bf16
+  static constexpr int BOX_C = BN * 64 * 2;    // [BN rows][64 cols] bf16
+  static constexpr int TILE_R = 128 * D * 2;
+  static constexpr int TILE_C = BN * D * 2;
+  static constexpr int ST1 = (D == 128 && BN == 128) ? 3 : 4;   // C1 ring slots
+  static constexpr int ST2 = (D == 128 && BN == 128) ? 2 : 4;   // C2 ring slots
   static constexpr int OFF_R1 = 0;
-  static constexpr int OFF_R2 = TILE_BYTES;
-  static constexpr int OFF_C1 = 2 * TILE_BYTES;
-  static constexpr int OFF_C2 = OFF_C1 + ST1 * TILE_BYTES;
-  static constexpr int SMEM_BYTES = OFF_C2 + ST2 * TILE_BYTES;
+  static constexpr int OFF_R2 = TILE_R;
+  static constexpr int OFF_C1 = 2 * TILE_R;
+  static constexpr int OFF_C2 = OFF_C1 + ST1 * TILE_C;
+  static constexpr int SMEM_BYTES = OFF_C2 + ST2 * TILE_C;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   static constexpr int TM_XS = 0;
-  static constexpr int TM_XDP = SPLIT_X ? 128 : 0;
-  static constexpr int TM_P = SPLIT_X ? 256 : 128;
-  static constexpr int TM_DS = TM_P + 64;
-  static constexpr int TM_A1 = TM_DS + 64;
-  static constexpr int TM_A2 = TM_A1 + D;
+  static constexpr int TM_XDP = BN;
+  static constexpr int TM_P = 2 * BN;
+  static constexpr int TM_DS = 2 * BN + BN / 2;
+  static constexpr int TM_A1 = 3 * BN;
+  static constexpr int TM_A2 = 3 * BN + D;
   static constexpr int TMEM_COLS = 512;
   static_assert(TM_A1 + (KV ? 2 : 1) * D <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_ALLOC <= 227 * 1024 - 1024, "shared memory budget");
   static constexpr int EPI_WARPS = 8;
-  static constexpr int ISSUERS = 2 + (SPLIT_X ? 1 : 0) + (KV ? 1 : 0);
+  static constexpr int ISSUERS = KV ? 4 : 3;
   static constexpr int THREADS = (EPI_WARPS + 1 + ISSUERS) * 32;
-  // Load both dP chunks at once when registers allow (fewer warps).
-  static constexpr bool DP_BOTH = THREADS <= 384;
 };
 
 template <int ST1, int ST2>
@@ -104,13 +103,13 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   volatile int* abort_flag = &bar.abort;
   constexpr int kProducerWarp = C::EPI_WARPS;
   constexpr int kSWarp = C::EPI_WARPS + 1;
-  constexpr int kDPWarp = C::SPLIT_X ? C::EPI_WARPS + 2 : -1;
-  constexpr int kA1Warp = C::EPI_WARPS + (C::SPLIT_X ? 3 : 2);
-  constexpr int kA2Warp = KV ? kA1Warp + 1 : -1;
+  constexpr int kDPWarp = C::EPI_WARPS + 2;
+  constexpr int kA1Warp = C::EPI_WARPS + 3;
+  constexpr int kA2Warp = KV ? C::EPI_WARPS + 4 : -1;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.r_full, 1);
-    mbar_init(&bar.r_empty, C::SPLIT_X ? 2 : 1);
+    mbar_init(&bar.r_empty, 2);  // S issuer (R1) and dP issuer (R2)
     for (int s = 0; s < C::ST1; ++s) {
       mbar_init(&bar.c1_full[s], 1);
       mbar_init(&bar.c1_empty[s], 2);  // S issuer and A1 issuer
@@ -148,17 +147,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   // Descriptor bases (built once, advanced by adding (bytes >> 4): the
   // start-address field is the low 14 bits and smem stays below 256 KB).
   const uint32_t sbase = smem_u32(smem);
-  constexpr uint64_t kTile = C::TILE_BYTES >> 4;
-  constexpr uint32_t idesc_x = idesc_bf16_f32(128, C::BN, false, false);
-
-  // X = R C^T over K = D (D/16 steps of K = 16), both operands K-major.
-  auto issue_x = [&](uint32_t d_tmem, uint64_t a0, uint64_t b0) {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t off = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-      mma_ss(d_tmem, a0 + off, b0 + off, idesc_x, kk > 0 ? 1u : 0u);
-    }
-  };
+  constexpr uint64_t kTileC = C::TILE_C >> 4;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------- producer
@@ -177,25 +166,25 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         const int n = load_len(lengths, item.bh / H, L);
         const int nb = ceil_div(n, C::BN);
         if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, ws, 201))) break;
-        mbar_arrive_expect_tx(&bar.r_full, 2 * C::TILE_BYTES);
+        mbar_arrive_expect_tx(&bar.r_full, 2 * C::TILE_R);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem + C::OFF_R1 + c * C::BOX_BYTES, &tm_r1, &bar.r_full, c * 64, item.blk * C::BM, item.bh);
-          tma_load_3d(smem + C::OFF_R2 + c * C::BOX_BYTES, &tm_r2, &bar.r_full, c * 64, item.blk * C::BM, item.bh);
+          tma_load_3d(smem + C::OFF_R1 + c * C::BOX_R, &tm_r1, &bar.r_full, c * 64, item.blk * C::BM, item.bh);
+          tma_load_3d(smem + C::OFF_R2 + c * C::BOX_R, &tm_r2, &bar.r_full, c * 64, item.blk * C::BM, item.bh);
         }
         r_last = static_cast<int>(rph);
         rph ^= 1;
         for (int j = 0; j < nb; ++j) {
           if (!(ok = mbar_wait(&bar.c1_empty[s1], p1 ^ 1, abort_flag, ws, 202))) break;
-          mbar_arrive_expect_tx(&bar.c1_full[s1], C::TILE_BYTES);
+          mbar_arrive_expect_tx(&bar.c1_full[s1], C::TILE_C);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + C::OFF_C1 + s1 * C::TILE_BYTES + c * C::BOX_BYTES, &tm_c1, &bar.c1_full[s1], c * 64,
+            tma_load_3d(smem + C::OFF_C1 + s1 * C::TILE_C + c * C::BOX_C, &tm_c1, &bar.c1_full[s1], c * 64,
                         j * C::BN, item.bh);
           c1_last[s1] = static_cast<int>(p1);
           if (++s1 == C::ST1) { s1 = 0; p1 ^= 1; }
           if (!(ok = mbar_wait(&bar.c2_empty[s2], p2 ^ 1, abort_flag, ws, 203))) break;
-          mbar_arrive_expect_tx(&bar.c2_full[s2], C::TILE_BYTES);
+          mbar_arrive_expect_tx(&bar.c2_full[s2], C::TILE_C);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + C::OFF_C2 + s2 * C::TILE_BYTES + c * C::BOX_BYTES, &tm_c2, &bar.c2_full[s2], c * 64,
+            tma_load_3d(smem + C::OFF_C2 + s2 * C::TILE_C + c * C::BOX_C, &tm_c2, &bar.c2_full[s2], c * 64,
                         j * C::BN, item.bh);
           c2_last[s2] = static_cast<int>(p2);
           if (++s2 == C::ST2) { s2 = 0; p2 ^= 1; }
@@ -212,14 +201,19 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       }
     }
   } else if (warp == kSWarp || warp == kDPWarp) {
-    // ------------------------- issuers of S (and, with one region, dP) into X
+    // ------------------------------------------ issuers of S = R1 C1^T, dP = R2 C2^T
     if (lane == 0) {
-      const bool is_dp = (warp == kDPWarp);  // separate dP issuer (SPLIT_X only)
-      const uint64_t d_r1 = smem_desc_sw128(sbase + C::OFF_R1, 16, 1024);
-      const uint64_t d_r2 = smem_desc_sw128(sbase + C::OFF_R2, 16, 1024);
-      const uint64_t d_c1 = smem_desc_sw128(sbase + C::OFF_C1, 16, 1024);
-      const uint64_t d_c2 = smem_desc_sw128(sbase + C::OFF_C2, 16, 1024);
-      uint32_t s1 = 0, p1 = 0, s2 = 0, p2 = 0, rph = 0, s_read_ph = 0, dp_read_ph = 0;
+      const bool is_dp = (warp == kDPWarp);
+      constexpr uint32_t idesc_x = idesc_bf16_f32(128, C::BN, false, false);
+      const uint64_t d_r = smem_desc_sw128(sbase + (is_dp ? C::OFF_R2 : C::OFF_R1), 16, 1024);
+      const uint64_t d_c = smem_desc_sw128(sbase + (is_dp ? C::OFF_C2 : C::OFF_C1), 16, 1024);
+      const uint32_t d_tmem = tmem + (is_dp ? C::TM_XDP : C::TM_XS);
+      const int slots = is_dp ? C::ST2 : C::ST1;
+      uint64_t* cfull = is_dp ? bar.c2_full : bar.c1_full;
+      uint64_t* cempty = is_dp ? bar.c2_empty : bar.c1_empty;
+      uint64_t* xfull = is_dp ? &bar.xdp_full : &bar.xs_full;
+      uint64_t* xread = is_dp ? &bar.xdp_read : &bar.xs_read;
+      uint32_t st = 0, cph = 0, rph = 0, read_ph = 0;
       bool ok = true;
       for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
         const Item item = load_item(ws, it);
@@ -228,40 +222,21 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         if (!(ok = mbar_wait(&bar.r_full, rph, abort_flag, ws, 211))) break;
         rph ^= 1;
         for (int j = 0; j < nb; ++j) {
-          if (!is_dp) {
-            // S(j): its region is free once the epilogue has copied out
-            // S(j-1) (separate regions) or dP(j-1) (one shared region).
-            if (!(ok = mbar_wait(&bar.c1_full[s1], p1, abort_flag, ws, 212))) break;
-            if (C::SPLIT_X) {
-              if (!(ok = mbar_wait(&bar.xs_read, s_read_ph ^ 1, abort_flag, ws, 213))) break;
-              s_read_ph ^= 1;
-            } else {
-              if (!(ok = mbar_wait(&bar.xdp_read, dp_read_ph ^ 1, abort_flag, ws, 213))) break;
-              dp_read_ph ^= 1;
-            }
-            tc_fence_after();
-            issue_x(tmem + C::TM_XS, d_r1, d_c1 + s1 * kTile);
-            mma_commit(&bar.xs_full);
-            mma_commit(&bar.c1_empty[s1]);
-            if (++s1 == C::ST1) { s1 = 0; p1 ^= 1; }
+          if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 212))) break;
+          // The region is free once the epilogue has copied out block j-1.
+          if (!(ok = mbar_wait(xread, read_ph ^ 1, abort_flag, ws, 213))) break;
+          read_ph ^= 1;
+          tc_fence_after();
+          const uint64_t b0 = d_c + st * kTileC;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // K = D in steps of 16
+            const uint64_t a_off = ((kk >> 2) * C::BOX_R + (kk & 3) * 32) >> 4;
+            const uint64_t b_off = ((kk >> 2) * C::BOX_C + (kk & 3) * 32) >> 4;
+            mma_ss(d_tmem, d_r + a_off, b0 + b_off, idesc_x, kk > 0 ? 1u : 0u);
           }
-          if (is_dp || !C::SPLIT_X) {
-            // dP(j): free once dP(j-1) (separate regions) or S(j) (one shared
-            // region) has been copied out.
-            if (!(ok = mbar_wait(&bar.c2_full[s2], p2, abort_flag, ws, 214))) break;
-            if (C::SPLIT_X) {
-              if (!(ok = mbar_wait(&bar.xdp_read, dp_read_ph ^ 1, abort_flag, ws, 215))) break;
-              dp_read_ph ^= 1;
-            } else {
-              if (!(ok = mbar_wait(&bar.xs_read, s_read_ph, abort_flag, ws, 215))) break;
-              s_read_ph ^= 1;
-            }
-            tc_fence_after();
-            issue_x(tmem + C::TM_XDP, d_r2, d_c2 + s2 * kTile);
-            mma_commit(&bar.xdp_full);
-            mma_commit(&bar.c2_empty[s2]);
-            if (++s2 == C::ST2) { s2 = 0; p2 ^= 1; }
-          }
+          mma_commit(xfull);
+          mma_commit(&cempty[st]);
+          if (++st == slots) { st = 0; cph ^= 1; }
           if (j + 1 == nb) mma_commit(&bar.r_empty);
         }
       }
@@ -274,8 +249,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     if (lane == 0) {
       const bool second = (warp == kA2Warp);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
-      // MN-major view of the C1 (A1) or C2 (A2) ring: rows = the K dimension.
-      const uint64_t d_cmn = smem_desc_sw128(sbase + (second ? C::OFF_C2 : C::OFF_C1), C::BOX_BYTES, 1024);
+      // MN-major view of the C1 (A1) or C2 (A2) ring: rows = the K dimension,
+      // the two 64-column halves of D BOX_C bytes apart.
+      const uint64_t d_cmn = smem_desc_sw128(sbase + (second ? C::OFF_C2 : C::OFF_C1), C::BOX_C, 1024);
       const int slots = second ? C::ST2 : C::ST1;
       uint64_t* cfull = second ? bar.c2_full : bar.c1_full;
       uint64_t* cempty = second ? bar.c2_empty : bar.c1_empty;
@@ -292,8 +268,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         const int nb = ceil_div(n, C::BN);
         for (int j = 0; ok && j < nb; ++j) {
           if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 231))) break;
-          const uint64_t b0 = d_cmn + st * kTile;
-          for (int q = 0; q < 4; ++q) {
+          const uint64_t b0 = d_cmn + st * kTileC;
+          for (int q = 0; q < C::NCH; ++q) {
             if (!(ok = mbar_wait(&full[q], fph[q], abort_flag, ws, 232))) break;
             fph[q] ^= 1;
             const bool first = (j == 0 && q == 0);
@@ -323,11 +299,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     }
   } else if (warp < C::EPI_WARPS) {
     // ------------------------------------------------------------- epilogue
-    const int g = warp >> 2;                      // column half: chunks 2g, 2g+1
+    constexpr int CPW = C::CPW;
+    const int g = warp >> 2;                      // chunks g*CPW .. g*CPW + CPW - 1
     const int r = ((warp & 3) << 5) + lane;       // row within the item = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
-    const uint32_t tXS = tmem + lane_off + C::TM_XS + g * 64;
-    const uint32_t tXDP = tmem + lane_off + C::TM_XDP + g * 64;
+    const uint32_t tXS = tmem + lane_off + C::TM_XS + g * CPW * 32;
+    const uint32_t tXDP = tmem + lane_off + C::TM_XDP + g * CPW * 32;
     constexpr float scale = Scale<D>::value;
     constexpr float half_scale = 0.5f * scale;
     uint32_t s_ph = 0, dp_ph = 0, free_ph = 0, aph = 0;
@@ -339,73 +316,68 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       const float half_bias = -0.5f * __logf(static_cast<float>(n));
       for (int j = 0; j < nb; ++j) {
         // ---- S -> P (fp32 kept in registers for dS), bf16 P for dV
-        float p[64];
-        uint32_t dp[2][32];
+        float p[CPW][32];
         {
-          uint32_t s0[32], s1[32];
+          uint32_t sv[CPW][32];
           if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, ws, 221))) break;
           s_ph ^= 1;
           tc_fence_after();
-          tmem_ld32x2(tXS, tXS + 32, s0, s1);
+#pragma unroll
+          for (int c = 0; c < CPW; ++c) tmem_ld32_async(tXS + 32 * c, sv[c]);
+#pragma unroll
+          for (int c = 0; c < CPW; ++c) tmem_ld_wait32(sv[c]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.xs_read);
-          if (!C::SPLIT_X) {
-            // One shared region: copy dP out as soon as it lands, so that the
-            // next block's S can be computed while this epilogue works.
-            if (!(ok = mbar_wait(&bar.xdp_full, dp_ph, abort_flag, ws, 222))) break;
-            dp_ph ^= 1;
-            tc_fence_after();
-            tmem_ld32x2(tXDP, tXDP + 32, dp[0], dp[1]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar.xdp_read);
-          }
-          const int valid = n - (j * C::BN + g * 64);  // columns < valid are real tokens
+          const int valid = n - (j * C::BN + g * CPW * 32);  // columns < valid are real tokens
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            p[e] = sigmoid_from_score(__uint_as_float(s0[e]), half_scale, half_bias);
-            p[32 + e] = sigmoid_from_score(__uint_as_float(s1[e]), half_scale, half_bias);
-          }
-          if (valid < 64) {
+          for (int c = 0; c < CPW; ++c)
 #pragma unroll
-            for (int e = 0; e < 64; ++e) p[e] = (e < valid) ? p[e] : 0.f;
-          }
+            for (int e = 0; e < 32; ++e) {
+              const float pe = sigmoid_from_score(__uint_as_float(sv[c][e]), half_scale, half_bias);
+              p[c][e] = (valid >= CPW * 32 || 32 * c + e < valid) ? pe : 0.f;
+            }
         }
         if (KV) {
           if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < CPW; ++c) {
             uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(p[32 * c + 2 * e], p[32 * c + 2 * e + 1]);
-            tmem_st16(tmem + lane_off + C::TM_P + (2 * g + c) * 16, pk);
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(p[c][2 * e], p[c][2 * e + 1]);
+            tmem_st16(tmem + lane_off + C::TM_P + (g * CPW + c) * 16, pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar.p_full[2 * g + c]);
+            if (lane == 0) mbar_arrive(&bar.p_full[g * CPW + c]);
           }
         }
-        // ---- dP -> dS = dP P (1 - P), bf16 dS for dQ / dK
-        if (C::SPLIT_X) {
-          if (!(ok = mbar_wait(&bar.xdp_full, dp_ph, abort_flag, ws, 222))) break;
-          dp_ph ^= 1;
-        }
-        if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, ws, 224))) break;
-        free_ph ^= 1;
+        // ---- dP -> dS = dP P (1 - P), bf16 dS for dQ / dK. The dK/dV kernel
+        // (fewer registers per thread) copies dP out one chunk at a time.
+        constexpr bool kDpAtOnce = !KV;
+        uint32_t dp[kDpAtOnce ? CPW : 1][32];
+        if (!(ok = mbar_wait(&bar.xdp_full, dp_ph, abort_flag, ws, 222))) break;
+        dp_ph ^= 1;
         tc_fence_after();
-        if (C::SPLIT_X && C::DP_BOTH) {
-          tmem_ld32x2(tXDP, tXDP + 32, dp[0], dp[1]);
+        if (kDpAtOnce) {
+#pragma unroll
+          for (int c = 0; c < CPW; ++c) tmem_ld32_async(tXDP + 32 * c, dp[kDpAtOnce ? c : 0]);
+#pragma unroll
+          for (int c = 0; c < CPW; ++c) tmem_ld_wait32(dp[kDpAtOnce ? c : 0]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.xdp_read);
         }
+        if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, ws, 224))) break;
+        free_ph ^= 1;
+        tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (C::SPLIT_X && !C::DP_BOTH) {
-            tmem_ld32(tXDP + 32 * c, dp[c]);
-            if (c == 1) {
+        for (int c = 0; c < CPW; ++c) {
+          uint32_t(&dpc)[32] = dp[kDpAtOnce ? c : 0];
+          if (!kDpAtOnce) {
+            tmem_ld32(tXDP + 32 * c, dpc);
+            if (c + 1 == CPW) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&bar.xdp_read);
@@ -414,16 +386,16 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float q0 = p[32 * c + 2 * e], q1 = p[32 * c + 2 * e + 1];
-            const float ds0 = __uint_as_float(dp[c][2 * e]) * (q0 - q0 * q0);
-            const float ds1 = __uint_as_float(dp[c][2 * e + 1]) * (q1 - q1 * q1);
+            const float q0 = p[c][2 * e], q1 = p[c][2 * e + 1];
+            const float ds0 = __uint_as_float(dpc[2 * e]) * (q0 - q0 * q0);
+            const float ds1 = __uint_as_float(dpc[2 * e + 1]) * (q1 - q1 * q1);
             pk[e] = pack_bf16x2(ds0, ds1);
           }
-          tmem_st16(tmem + lane_off + C::TM_DS + (2 * g + c) * 16, pk);
+          tmem_st16(tmem + lane_off + C::TM_DS + (g * CPW + c) * 16, pk);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bar.ds_full[2 * g + c]);
+          if (lane == 0) mbar_arrive(&bar.ds_full[g * CPW + c]);
         }
       }
       if (!ok) break;
@@ -436,20 +408,23 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       const size_t row_off = (static_cast<size_t>(item.bh) * L + row) * D;
       // 32-column chunks of the accumulators: A1 (-> out1, times scale), then
       // A2 (-> out2) for dK/dV; each half of the warps takes every other
-      // chunk. All of a thread's chunks are copied out first, so the
+      // chunk. Each chunk is copied out and packed to bf16 at once, so the
       // accumulators are released before the (slower) global stores.
       constexpr int kChunks = (KV ? 2 : 1) * (D / 32);
       constexpr int kPer = kChunks / 2;
-      uint32_t v[kPer][32];
+      uint32_t packed[kPer][16];
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
         const int c = g + 2 * i;
         const bool second = c >= D / 32;
         const int col = (second ? c - D / 32 : c) * 32;
-        tmem_ld32_async(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v[i]);
-      }
+        const float mul = (second ? 1.0f : scale) * (valid_row ? 1.0f : 0.0f);
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v);
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) tmem_ld_wait32(v[i]);
+        for (int e = 0; e < 16; ++e)
+          packed[i][e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.acc_empty);
@@ -459,9 +434,15 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const int c = g + 2 * i;
           const bool second = c >= D / 32;
           const int col = (second ? c - D / 32 : c) * 32;
-          __nv_bfloat16* dst = (second ? out2 : out1) + row_off + col;
-          if (valid_row) store_row32(dst, v[i], second ? 1.0f : scale);
-          else store_zero32(dst);
+          uint4* dst = reinterpret_cast<uint4*>((second ? out2 : out1) + row_off + col);
+          if (valid_row) {
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4)
+              dst[w4] = make_uint4(packed[i][4 * w4], packed[i][4 * w4 + 1], packed[i][4 * w4 + 2],
+                                   packed[i][4 * w4 + 3]);
+          } else {
+            store_zero32((second ? out2 : out1) + row_off + col);
+          }
         }
       }
     }

@@ -26,6 +26,10 @@ constexpr int kMaxLen = 1 << 20;       // Lmax bound (TMA coordinates are int32)
 
 __host__ __device__ constexpr int item_rows(int kind) { return kind == kKindFwd ? kFwdItemRows : kBwdItemRows; }
 
+// Columns per block streamed by a backward kernel: 128, except 64 for dK/dV
+// with d = 128 (its TMEM budget).
+__host__ __device__ constexpr int bwd_col_block(bool kv, int d) { return (kv && d == 128) ? 64 : 128; }
+
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Valid length of sequence b, or 0 if the caller's value is outside [0, L]
