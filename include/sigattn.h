@@ -148,6 +148,14 @@ SIGATTN_API int sigattn_fwd_noalloc(const void* q, const void* k, const void* v,
  * calling thread (static, thread-local; "no error" if none yet). */
 SIGATTN_API const char* sigattn_last_error(void);
 
+/* Diagnostic for the failure path: enqueue a one-warp kernel whose bounded
+ * wait on an mbarrier that nothing arrives on must give up after limit_us
+ * microseconds (1 .. 10^7). The kernel records SIGATTN_ERR_TIMEOUT with site
+ * 901 in the workspace header, exactly as a compute kernel's expired wait
+ * does, and returns normally (the context stays usable). Needs only the
+ * 256-byte header of a workspace. */
+SIGATTN_API int sigattn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int limit_us, void* stream);
+
 /* Synchronise `stream`, read the workspace's sticky error word, clear it and
  * return it (SIGATTN_OK if no kernel reported a problem). If `site` is not
  * NULL it receives a code naming the failing check or wait (0 if none). */

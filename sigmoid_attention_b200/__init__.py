@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "SigattnError", "library", "library_path", "sigattn_version", "sigattn_status_str", "sigattn_block_rows",
     "sigattn_workspace_size", "sigattn_fwd", "sigattn_fwd_noalloc", "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
-    "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "read_plan", "make_workspace", "forward", "backward",
+    "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
     "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
 ]
 
@@ -75,6 +75,8 @@ def library():
         lib.sigattn_plan_host.argtypes = [_vp] + [_i] * 4 + [_vp, _i, ctypes.POINTER(_i)]
         lib.sigattn_fwd_noalloc.restype = _i
         lib.sigattn_fwd_noalloc.argtypes = [_vp] * 5 + [_i] * 4 + [_vp, _vp]
+        lib.sigattn_selftest_wait_timeout.restype = _i
+        lib.sigattn_selftest_wait_timeout.argtypes = [_vp, _sz, _i, _vp]
         lib.sigattn_last_error.restype = ctypes.c_char_p
         lib.sigattn_last_error.argtypes = []
         lib.sigattn_read_error.restype = _i
@@ -191,6 +193,12 @@ def sigattn_plan_host(lengths, H: int, Lmax: int, kind: int) -> torch.Tensor:
     _check("sigattn_plan_host", lib.sigattn_plan_host(lens.data_ptr(), B, H, Lmax, kind, out.data_ptr(),
                                                       count.value, ctypes.byref(count)))
     return out[:count.value]
+
+
+def sigattn_selftest_wait_timeout(workspace, limit_us: int = 20000, stream=None) -> None:
+    """Enqueue the diagnostic kernel whose bounded wait must expire (see the header)."""
+    _check("sigattn_selftest_wait_timeout", library().sigattn_selftest_wait_timeout(
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), int(limit_us), _stream_ptr(stream)))
 
 
 def sigattn_last_error() -> str:

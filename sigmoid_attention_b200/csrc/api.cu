@@ -13,6 +13,7 @@ namespace sigattn {
 cudaError_t launch_prep(const int* lengths, int B, int H, int L, int d, int kind, int* ws, void* out0, void* out1,
                         int num_sms, cudaStream_t stream);
 int plan_host(const int* lengths, int B, int H, int L, int kind, int* out, int cap);
+cudaError_t launch_selftest_timeout(int* ws, unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                        const int* lengths, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
@@ -246,6 +247,18 @@ int sigattn_plan_host(const int32_t* lengths_host, int B, int H, int Lmax, int k
 }
 
 const char* sigattn_last_error(void) { return g_last_error; }
+
+int sigattn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int limit_us, void* stream) {
+  if (!aligned16(workspace) || workspace_bytes < static_cast<size_t>(kHeaderWords) * 4 || limit_us < 1 ||
+      limit_us > 10000000)
+    return SIGATTN_ERR_INVALID_ARG;
+  DeviceInfo info;
+  if (!device_info(&info)) return cuda_status(cudaErrorUnknown);
+  if (!info.supported) return SIGATTN_ERR_UNSUPPORTED;
+  return cuda_status(launch_selftest_timeout(static_cast<int*>(workspace),
+                                             static_cast<unsigned long long>(limit_us) * 1000ull,
+                                             static_cast<cudaStream_t>(stream)));
+}
 
 int sigattn_read_error(void* workspace, int* site, void* stream) {
   if (!aligned16(workspace)) return SIGATTN_ERR_INVALID_ARG;

@@ -14,9 +14,9 @@ namespace sigattn {
 //  * forward: 256 query rows (two 128-row query tiles sharing each K/V block),
 //  * dQ:      128 query rows,
 //  * dK/dV:   128 key rows.
-// Every inner loop walks blocks of 128 columns (keys for forward/dQ, queries
-// for dK/dV) up to ceil(n/128), so fully padded blocks are never touched on
-// either side.
+// Every inner loop walks blocks of columns (keys for forward/dQ, queries for
+// dK/dV; 128 wide, 64 for dK/dV at d = 128) only up to the last block holding
+// a valid token, so fully padded blocks are never touched on either side.
 enum Kind : int { kKindFwd = 0, kKindDq = 1, kKindDkdv = 2 };
 constexpr int kFwdItemRows = 256;
 constexpr int kBwdItemRows = 128;

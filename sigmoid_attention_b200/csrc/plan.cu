@@ -7,7 +7,7 @@
 // host never has to read the lengths back:
 //
 //   * one work item per (b, h, row block) whose first row is < n_b; the
-//     compute kernels walk column blocks only up to ceil(n_b / 128);
+//     compute kernels walk column blocks only up to ceil(n_b / block width);
 //   * sequences are ordered longest first (stable in b), and a persistent
 //     compute grid takes items round-robin, which spreads the long items over
 //     all SMs first (longest-processing-time-first order);
@@ -122,6 +122,27 @@ cudaError_t launch_prep(const int* lengths, int B, int H, int L, int d, int kind
   prep_kernel<<<grid, 1024, smem, stream>>>(lengths, B, H, L, d, item_rows(kind), ws,
                                             static_cast<__nv_bfloat16*>(out0),
                                             static_cast<__nv_bfloat16*>(out1));
+  return cudaGetLastError();
+}
+
+// Diagnostic: one warp waits, with a bounded wait, on an mbarrier that nothing
+// arrives on. The wait must give up after `limit_ns` and record the timeout in
+// the workspace header exactly as a compute kernel's wait would (site 901).
+__global__ void selftest_timeout_kernel(int* ws, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, ws, 901, limit_ns);
+  __syncthreads();
+}
+
+cudaError_t launch_selftest_timeout(int* ws, unsigned long long limit_ns, cudaStream_t stream) {
+  selftest_timeout_kernel<<<1, 32, 0, stream>>>(ws, limit_ns);
   return cudaGetLastError();
 }
 

@@ -188,3 +188,17 @@ def test_autograd_function_matches_direct_calls():
     assert torch.equal(qd.grad.float().cpu(), ref_dq)
     assert torch.equal(kd.grad.float().cpu(), ref_dk)
     assert torch.equal(vd.grad.float().cpu(), ref_dv)
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives():
+    """The failure path: a wait that nothing satisfies gives up after its limit,
+    records SIGATTN_ERR_TIMEOUT (site 901) in the workspace and leaves the
+    context usable for the next call."""
+    B, H, L, d = 1, 2, 256, 64
+    ws = sa.make_workspace(B, H, L, d)
+    sa.sigattn_selftest_wait_timeout(ws, limit_us=20000)
+    assert sa.sigattn_read_error(ws) == (4, 901)
+    assert sa.sigattn_read_error(ws) == (0, 0)  # sticky until read, then cleared
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 51)
+    o, *_ = run_gpu(q, k, v, dout, [200])
+    assert rel_l2(o, oracle.forward(q, k, v, [200])) <= FWD_REL
