@@ -66,6 +66,10 @@ struct BwdCfg {
   static constexpr int TM_A2 = 3 * BN + D;
   static constexpr int TMEM_COLS = 512;
   static_assert(TM_A1 + (KV ? 2 : 1) * D <= TMEM_COLS, "TMEM budget");
+  // A second dP region where the columns allow (dK/dV at D = 128): the dP
+  // products of block j+1 need not wait for the epilogue to copy out dP(j).
+  static constexpr int TM_XDP1 = TM_A1 + (KV ? 2 : 1) * D;
+  static constexpr int NXDP = (TM_XDP1 + BN <= TMEM_COLS) ? 2 : 1;
   static_assert(SMEM_ALLOC <= 227 * 1024 - 1024, "shared memory budget");
   static constexpr int EPI_WARPS = 8;
   static constexpr int ISSUERS = KV ? 4 : 3;
@@ -77,8 +81,8 @@ struct BwdBarriers {
   uint64_t r_full, r_empty;
   uint64_t c1_full[ST1], c1_empty[ST1];
   uint64_t c2_full[ST2], c2_empty[ST2];
-  uint64_t xs_full, xdp_full;      // S / dP of the current block are in TMEM
-  uint64_t xs_read, xdp_read;      // the epilogue has copied S / dP out
+  uint64_t xs_full, xdp_full[2];   // S / dP of the current block are in TMEM
+  uint64_t xs_read, xdp_read[2];   // the epilogue has copied S / dP out (per dP region)
   uint64_t p_full[4], ds_full[4];  // bf16 P / dS of a 32-column chunk written
   uint64_t p_free, ds_free;        // the accumulation products of a block have read P / dS
   uint64_t acc_full, acc_empty;
@@ -119,9 +123,11 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       mbar_init(&bar.c2_empty[s], KV ? 2 : 1);  // dP issuer (and A2 issuer)
     }
     mbar_init(&bar.xs_full, 1);
-    mbar_init(&bar.xdp_full, 1);
     mbar_init(&bar.xs_read, C::EPI_WARPS);
-    mbar_init(&bar.xdp_read, C::EPI_WARPS);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar.xdp_full[b], 1);
+      mbar_init(&bar.xdp_read[b], C::EPI_WARPS);
+    }
     for (int q = 0; q < 4; ++q) {
       mbar_init(&bar.p_full[q], 4);
       mbar_init(&bar.ds_full[q], 4);
@@ -207,13 +213,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       constexpr uint32_t idesc_x = idesc_bf16_f32(128, C::BN, false, false);
       const uint64_t d_r = smem_desc_sw128(sbase + (is_dp ? C::OFF_R2 : C::OFF_R1), 16, 1024);
       const uint64_t d_c = smem_desc_sw128(sbase + (is_dp ? C::OFF_C2 : C::OFF_C1), 16, 1024);
-      const uint32_t d_tmem = tmem + (is_dp ? C::TM_XDP : C::TM_XS);
+      const int nbuf = is_dp ? C::NXDP : 1;     // regions this issuer rotates through
       const int slots = is_dp ? C::ST2 : C::ST1;
       uint64_t* cfull = is_dp ? bar.c2_full : bar.c1_full;
       uint64_t* cempty = is_dp ? bar.c2_empty : bar.c1_empty;
-      uint64_t* xfull = is_dp ? &bar.xdp_full : &bar.xs_full;
-      uint64_t* xread = is_dp ? &bar.xdp_read : &bar.xs_read;
-      uint32_t st = 0, cph = 0, rph = 0, read_ph = 0;
+      uint32_t st = 0, cph = 0, rph = 0, xb = 0;
+      uint32_t read_ph[2] = {0, 0};
       bool ok = true;
       for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
         const Item item = load_item(ws, it);
@@ -223,9 +228,13 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         rph ^= 1;
         for (int j = 0; j < nb; ++j) {
           if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 212))) break;
-          // The region is free once the epilogue has copied out block j-1.
-          if (!(ok = mbar_wait(xread, read_ph ^ 1, abort_flag, ws, 213))) break;
-          read_ph ^= 1;
+          // The region is free once the epilogue has copied out the block that
+          // last used it (block j-1, or j-2 with two dP regions).
+          uint64_t* xread = is_dp ? &bar.xdp_read[xb] : &bar.xs_read;
+          uint64_t* xfull = is_dp ? &bar.xdp_full[xb] : &bar.xs_full;
+          const uint32_t d_tmem = tmem + (is_dp ? (xb ? C::TM_XDP1 : C::TM_XDP) : C::TM_XS);
+          if (!(ok = mbar_wait(xread, read_ph[xb] ^ 1, abort_flag, ws, 213))) break;
+          read_ph[xb] ^= 1;
           tc_fence_after();
           const uint64_t b0 = d_c + st * kTileC;
 #pragma unroll
@@ -237,6 +246,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           mma_commit(xfull);
           mma_commit(&cempty[st]);
           if (++st == slots) { st = 0; cph ^= 1; }
+          if (++xb == static_cast<uint32_t>(nbuf)) xb = 0;
           if (j + 1 == nb) mma_commit(&bar.r_empty);
         }
       }
@@ -304,10 +314,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     const int r = ((warp & 3) << 5) + lane;       // row within the item = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
     const uint32_t tXS = tmem + lane_off + C::TM_XS + g * CPW * 32;
-    const uint32_t tXDP = tmem + lane_off + C::TM_XDP + g * CPW * 32;
+    const uint32_t tXDP0 = tmem + lane_off + C::TM_XDP + g * CPW * 32;
+    const uint32_t tXDP1 = tmem + lane_off + C::TM_XDP1 + g * CPW * 32;
     constexpr float scale = Scale<D>::value;
     constexpr float half_scale = 0.5f * scale;
-    uint32_t s_ph = 0, dp_ph = 0, free_ph = 0, aph = 0;
+    uint32_t s_ph = 0, free_ph = 0, aph = 0, xb = 0;
+    uint32_t dp_ph[2] = {0, 0};
     bool ok = true;
     for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
       const Item item = load_item(ws, it);
@@ -357,8 +369,11 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         // (fewer registers per thread) copies dP out one chunk at a time.
         constexpr bool kDpAtOnce = !KV;
         uint32_t dp[kDpAtOnce ? CPW : 1][32];
-        if (!(ok = mbar_wait(&bar.xdp_full, dp_ph, abort_flag, ws, 222))) break;
-        dp_ph ^= 1;
+        const uint32_t tXDP = xb ? tXDP1 : tXDP0;
+        uint64_t* xdp_read = &bar.xdp_read[xb];
+        if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, ws, 222))) break;
+        dp_ph[xb] ^= 1;
+        if (++xb == static_cast<uint32_t>(C::NXDP)) xb = 0;
         tc_fence_after();
         if (kDpAtOnce) {
 #pragma unroll
@@ -367,7 +382,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           for (int c = 0; c < CPW; ++c) tmem_ld_wait32(dp[kDpAtOnce ? c : 0]);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bar.xdp_read);
+          if (lane == 0) mbar_arrive(xdp_read);
         }
         if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, ws, 224))) break;
         free_ph ^= 1;
@@ -380,7 +395,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
             if (c + 1 == CPW) {
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(&bar.xdp_read);
+              if (lane == 0) mbar_arrive(xdp_read);
             }
           }
           uint32_t pk[16];
