@@ -82,7 +82,7 @@ SIGATTN_API const char* sigattn_status_str(int status);
 SIGATTN_API int sigattn_block_rows(int kind);
 
 /* Bytes of workspace needed for any of the three calls with these sizes
- * (a 256-byte header plus one 8-byte entry per possible work item).
+ * (a 256-byte header plus one 16-byte entry per possible work item).
  * Returns 0 if the sizes are out of range. */
 SIGATTN_API size_t sigattn_workspace_size(int B, int H, int Lmax, int d);
 
@@ -105,9 +105,9 @@ SIGATTN_API int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, co
 
 /* Run only the ragged tile scheduler for `kind` on the device: afterwards the
  * workspace holds, at byte offset 8, the item count (int32), and at byte
- * offset 256, `count` pairs (int32 bh = b*H + h, int32 block index), ordered
- * longest sequence first (ties in batch order), heads ascending, blocks
- * ascending. Only blocks whose first row is < n_b appear (sec. 2C: fully
+ * offset 256, `count` entries of four int32 (bh = b*H + h, block index, the
+ * valid length n_b, 0), ordered longest sequence first (ties in batch order),
+ * heads ascending, blocks ascending. Only blocks whose first row is < n_b appear (sec. 2C: fully
  * padded blocks are skipped). */
 SIGATTN_API int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind, void* workspace,
                  size_t workspace_bytes, void* stream);
@@ -131,7 +131,7 @@ SIGATTN_API int sigattn_plan_host(const int32_t* lengths_host, int B, int H, int
  *    part of the library's device image, held on every GPU that loads the
  *    library until the process exits. It calls no cudaMalloc/cudaFree.
  *  - Size limit: sigattn_workspace_size(B, H, Lmax, d) must not exceed
- *    SIGATTN_NOALLOC_SCRATCH_BYTES, i.e. B*H*ceil(Lmax/128) <= 131040 work
+ *    SIGATTN_NOALLOC_SCRATCH_BYTES, i.e. B*H*ceil(Lmax/128) <= 65520 work
  *    items; larger problems return SIGATTN_ERR_UNSUPPORTED (message in
  *    sigattn_last_error) before anything is enqueued.
  *  - The first call on a device looks up the array's device address

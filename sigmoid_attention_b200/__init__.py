@@ -178,7 +178,7 @@ def read_plan(workspace: torch.Tensor) -> torch.Tensor:
     """The (bh, block) pairs the last plan wrote, as an int32 CPU tensor [count, 2]."""
     words = workspace.view(torch.int32).cpu()
     count = int(words[2])
-    return words[64:64 + 2 * count].view(count, 2).clone()
+    return words[64:64 + 4 * count].view(count, 4)[:, :2].clone()
 
 
 def sigattn_plan_host(lengths, H: int, Lmax: int, kind: int) -> torch.Tensor:

@@ -10,18 +10,19 @@
 #include "common.cuh"
 
 namespace sigattn {
-cudaError_t launch_prep(const int* lengths, int B, int H, int L, int d, int kind, int* ws, void* out0, void* out1,
+cudaError_t launch_prep(const int* lengths, int B, int H, int L, int kind, int* ws, cudaStream_t stream);
+cudaError_t launch_fill(const int* lengths, int B, int H, int L, int d, int kind, void* out0, void* out1,
                         int num_sms, cudaStream_t stream);
 int plan_host(const int* lengths, int B, int H, int L, int kind, int* out, int cap);
 cudaError_t launch_selftest_timeout(int* ws, unsigned long long limit_ns, cudaStream_t stream);
-cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                       const int* lengths, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream);
+cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
+                       int B, int H, int L, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                          const CUtensorMap& tv, void* dq, const int* lengths, int* ws, int B, int H, int L,
-                          int num_sms, cudaStream_t stream);
+                          const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L, int num_sms,
+                          cudaStream_t stream);
 cudaError_t launch_bwd_dkdv(int d, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                            const CUtensorMap& tdo, void* dk, void* dv, const int* lengths, int* ws, int B, int H,
-                            int L, int num_sms, cudaStream_t stream);
+                            const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int L, int num_sms,
+                            cudaStream_t stream);
 void set_last_error(const char* msg);
 }  // namespace sigattn
 
@@ -166,7 +167,7 @@ int sigattn_block_rows(int kind) {
 
 size_t sigattn_workspace_size(int B, int H, int Lmax, int d) {
   if (check_sizes(B, H, Lmax, d) != SIGATTN_OK) return 0;
-  return static_cast<size_t>(kHeaderWords) * 4 + static_cast<size_t>(max_items(B, H, Lmax)) * 8;
+  return static_cast<size_t>(kHeaderWords) * 4 + static_cast<size_t>(max_items(B, H, Lmax)) * 16;
 }
 
 int sigattn_fwd(const void* q, const void* k, const void* v, void* o, const int32_t* lengths, int B, int H,
@@ -180,9 +181,10 @@ int sigattn_fwd(const void* q, const void* k, const void* v, void* o, const int3
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, B, H, Lmax, d, SIGATTN_KIND_FWD, ws, o, nullptr, info.num_sms, s));
+  st = cuda_status(launch_prep(lengths, B, H, Lmax, SIGATTN_KIND_FWD, ws, s));
+  if (st == SIGATTN_OK) st = cuda_status(launch_fwd(d, tq, tk, tv, o, ws, B, H, Lmax, info.num_sms, s));
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_fwd(d, tq, tk, tv, o, lengths, ws, B, H, Lmax, info.num_sms, s));
+  return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_FWD, o, nullptr, info.num_sms, s));
 }
 
 int sigattn_bwd_dq(const void* q, const void* k, const void* v, const void* dout, void* dq, const int32_t* lengths,
@@ -198,9 +200,10 @@ int sigattn_bwd_dq(const void* q, const void* k, const void* v, const void* dout
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, B, H, Lmax, d, SIGATTN_KIND_DQ, ws, dq, nullptr, info.num_sms, s));
+  st = cuda_status(launch_prep(lengths, B, H, Lmax, SIGATTN_KIND_DQ, ws, s));
+  if (st == SIGATTN_OK) st = cuda_status(launch_bwd_dq(d, tq, tdo, tk, tv, dq, ws, B, H, Lmax, info.num_sms, s));
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_bwd_dq(d, tq, tdo, tk, tv, dq, lengths, ws, B, H, Lmax, info.num_sms, s));
+  return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_DQ, dq, nullptr, info.num_sms, s));
 }
 
 int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
@@ -220,9 +223,11 @@ int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* do
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, B, H, Lmax, d, SIGATTN_KIND_DKDV, ws, dk, dv, info.num_sms, s));
+  st = cuda_status(launch_prep(lengths, B, H, Lmax, SIGATTN_KIND_DKDV, ws, s));
+  if (st == SIGATTN_OK)
+    st = cuda_status(launch_bwd_dkdv(d, tk, tv, tq, tdo, dk, dv, ws, B, H, Lmax, info.num_sms, s));
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_bwd_dkdv(d, tk, tv, tq, tdo, dk, dv, lengths, ws, B, H, Lmax, info.num_sms, s));
+  return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_DKDV, dk, dv, info.num_sms, s));
 }
 
 int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind, void* workspace,
@@ -231,8 +236,8 @@ int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind
   DeviceInfo info;
   int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_prep(lengths, B, H, Lmax, d, kind, static_cast<int*>(workspace), nullptr, nullptr,
-                                 info.num_sms, static_cast<cudaStream_t>(stream)));
+  return cuda_status(
+      launch_prep(lengths, B, H, Lmax, kind, static_cast<int*>(workspace), static_cast<cudaStream_t>(stream)));
 }
 
 int sigattn_plan_host(const int32_t* lengths_host, int B, int H, int Lmax, int kind, int32_t* items_out, int cap,

@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_r1, const __grid_constant__ CUtensorMap tm_r2,
                const __grid_constant__ CUtensorMap tm_c1, const __grid_constant__ CUtensorMap tm_c2,
                __nv_bfloat16* __restrict__ out1, __nv_bfloat16* __restrict__ out2,
-               const int* __restrict__ lengths, int* __restrict__ ws, int H, int L) {
+               int* __restrict__ ws, int H, int L) {
   using C = BwdCfg<D, KV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ BwdBarriers<C::ST1, C::ST2> bar;
@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = &bar.abort;
+  grid_dep_launch();  // the padded-row fill kernel may start beside this one
   constexpr int kProducerWarp = C::EPI_WARPS;
   constexpr int kSWarp = C::EPI_WARPS + 1;
   constexpr int kDPWarp = C::EPI_WARPS + 2;
@@ -144,6 +145,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     tmem_alloc(&bar.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
+  // The plan is written by the kernel before this one in the stream.
+  grid_dep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -167,9 +170,11 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       for (int s = 0; s < C::ST1; ++s) c1_last[s] = -1;
       for (int s = 0; s < C::ST2; ++s) c2_last[s] = -1;
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
-        const Item item = load_item(ws, it);
-        const int n = load_len(lengths, item.bh / H, L);
+      Item nxt = load_item_or_empty(ws, item_slot(0), count);
+      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
+        const Item item = nxt;
+        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+        const int n = item.n;
         const int nb = ceil_div(n, C::BN);
         if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, ws, 201))) break;
         mbar_arrive_expect_tx(&bar.r_full, 2 * C::TILE_R);
@@ -220,9 +225,11 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       uint32_t st = 0, cph = 0, rph = 0, xb = 0;
       uint32_t read_ph[2] = {0, 0};
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
-        const Item item = load_item(ws, it);
-        const int n = load_len(lengths, item.bh / H, L);
+      Item nxt = load_item_or_empty(ws, item_slot(0), count);
+      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
+        const Item item = nxt;
+        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+        const int n = item.n;
         const int nb = ceil_div(n, C::BN);
         if (!(ok = mbar_wait(&bar.r_full, rph, abort_flag, ws, 211))) break;
         rph ^= 1;
@@ -272,9 +279,11 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       uint32_t st = 0, cph = 0, aph = 0;
       uint32_t fph[4] = {0, 0, 0, 0};
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
-        const Item item = load_item(ws, it);
-        const int n = load_len(lengths, item.bh / H, L);
+      Item nxt = load_item_or_empty(ws, item_slot(0), count);
+      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
+        const Item item = nxt;
+        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+        const int n = item.n;
         const int nb = ceil_div(n, C::BN);
         for (int j = 0; ok && j < nb; ++j) {
           if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 231))) break;
@@ -321,9 +330,11 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     uint32_t s_ph = 0, free_ph = 0, aph = 0, xb = 0;
     uint32_t dp_ph[2] = {0, 0};
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
-      const Item item = load_item(ws, it);
-      const int n = load_len(lengths, item.bh / H, L);
+    Item nxt = load_item_or_empty(ws, item_slot(0), count);
+    for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
+      const Item item = nxt;
+      nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+      const int n = item.n;
       const int nb = ceil_div(n, C::BN);
       const float half_bias = -0.5f * __logf(static_cast<float>(n));
       for (int j = 0; j < nb; ++j) {
@@ -473,8 +484,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
 
 template <int D, bool KV>
 cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
-                            const CUtensorMap& c2, void* out1, void* out2, const int* lengths, int* ws, int B,
-                            int H, int L, int num_sms, cudaStream_t stream) {
+                            const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
+                            cudaStream_t stream) {
   using C = BwdCfg<D, KV>;
   static bool configured[64] = {};
   int dev = 0;
@@ -487,23 +498,22 @@ cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const 
   }
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kBwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
-  bwd_kernel<D, KV><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(
-      r1, r2, c1, c2, static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), lengths, ws, H, L);
-  return cudaGetLastError();
+  return launch_programmatic(bwd_kernel<D, KV>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2, c1, c2,
+                             static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), ws, H, L);
 }
 
 cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                          const CUtensorMap& tv, void* dq, const int* lengths, int* ws, int B, int H, int L,
-                          int num_sms, cudaStream_t stream) {
-  if (d == 64) return launch_bwd_impl<64, false>(tq, tdo, tk, tv, dq, nullptr, lengths, ws, B, H, L, num_sms, stream);
-  return launch_bwd_impl<128, false>(tq, tdo, tk, tv, dq, nullptr, lengths, ws, B, H, L, num_sms, stream);
+                          const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L, int num_sms,
+                          cudaStream_t stream) {
+  if (d == 64) return launch_bwd_impl<64, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, num_sms, stream);
+  return launch_bwd_impl<128, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, num_sms, stream);
 }
 
 cudaError_t launch_bwd_dkdv(int d, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                            const CUtensorMap& tdo, void* dk, void* dv, const int* lengths, int* ws, int B, int H,
-                            int L, int num_sms, cudaStream_t stream) {
-  if (d == 64) return launch_bwd_impl<64, true>(tk, tv, tq, tdo, dk, dv, lengths, ws, B, H, L, num_sms, stream);
-  return launch_bwd_impl<128, true>(tk, tv, tq, tdo, dk, dv, lengths, ws, B, H, L, num_sms, stream);
+                            const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int L, int num_sms,
+                            cudaStream_t stream) {
+  if (d == 64) return launch_bwd_impl<64, true>(tk, tv, tq, tdo, dk, dv, ws, B, H, L, num_sms, stream);
+  return launch_bwd_impl<128, true>(tk, tv, tq, tdo, dk, dv, ws, B, H, L, num_sms, stream);
 }
 
 }  // namespace sigattn

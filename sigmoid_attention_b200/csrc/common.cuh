@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
@@ -39,14 +40,33 @@ __device__ __forceinline__ int load_len(const int* lengths, int b, int L) {
   return (n < 0 || n > L) ? 0 : n;
 }
 
+// One work item as the plan stores it: 16 bytes {b * H + h, row block, n_b, 0},
+// so a kernel learns the item and its sequence's valid length from one load.
 struct Item {
   int bh;   // b * H + h
   int blk;  // row-block index within the slice
+  int n;    // valid length of sequence b
 };
 
 __device__ __forceinline__ Item load_item(const int* ws, int idx) {
-  const int2 v = reinterpret_cast<const int2*>(ws + kHeaderWords)[idx];
-  return Item{v.x, v.y};
+  const int4 v = reinterpret_cast<const int4*>(ws + kHeaderWords)[idx];
+  return Item{v.x, v.y, v.z};
+}
+
+// Index of the item a persistent CTA takes in its round r. The plan lists the
+// items longest first; dealing them out in serpentine order (CTAs 0..G-1,
+// then G-1..0, ...) evens out the per-CTA totals better than plain
+// round-robin, which gives CTA 0 the longest item of every round. Increases
+// with r, so a CTA is done at its first index >= count.
+__device__ __forceinline__ int item_slot(int r) {
+  const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  return r * g + ((r & 1) ? g - 1 - b : b);
+}
+
+// The item at `idx` (or an empty one past the end).
+// Loaded one item ahead, so the load's latency is off the item boundary.
+__device__ __forceinline__ Item load_item_or_empty(const int* ws, int idx, int count) {
+  return idx < count ? load_item(ws, idx) : Item{0, 0, 0};
 }
 
 // 1/sqrt(d) for the supported head sizes.
@@ -86,6 +106,25 @@ __device__ __forceinline__ void store_zero32(__nv_bfloat16* dst) {
   uint4* p = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int q = 0; q < 4; ++q) p[q] = make_uint4(0, 0, 0, 0);
+}
+
+// Launch `kernel` so that it may start while the previous kernel in `stream` is
+// still running (programmatic stream serialization). The kernel calls
+// grid_dep_wait() before it touches anything that earlier kernel writes.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_programmatic(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace sigattn

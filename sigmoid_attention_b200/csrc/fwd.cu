@@ -70,7 +70,7 @@ template <int D>
 __global__ void __launch_bounds__((16 + 3) * 32, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-               const int* __restrict__ lengths, int* __restrict__ ws, int H, int L) {
+               int* __restrict__ ws, int H, int L) {
   using C = FwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ FwdBarriers<C::KST, C::VST> bar;
@@ -82,6 +82,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = &bar.abort;
+  grid_dep_launch();  // the padded-row fill kernel may start beside this one
 
   if (threadIdx.x == 0) {
     // "empty" barriers take one arrival from each of the two issuers
@@ -108,6 +109,8 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     tmem_alloc(&bar.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
+  // The plan is written by the kernel before this one in the stream.
+  grid_dep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -127,9 +130,11 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       for (int s = 0; s < C::KST; ++s) k_last[s] = -1;
       for (int s = 0; s < C::VST; ++s) v_last[s] = -1;
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
-        const Item item = load_item(ws, it);
-        const int n = load_len(lengths, item.bh / H, L);
+      Item nxt = load_item_or_empty(ws, item_slot(0), count);
+      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
+        const Item item = nxt;
+        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+        const int n = item.n;
         const int row0 = item.blk * (C::BM * C::NQ);
         const int ntiles = (row0 + C::BM < n) ? 2 : 1;
         const int nkb = ceil_div(n, C::BN);
@@ -206,9 +211,12 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       auto advance_k = [&]() { if (++kst == C::KST) { kst = 0; kph ^= 1; } };
       auto advance_v = [&]() { if (++vst == C::VST) { vst = 0; vph ^= 1; } };
 
-      for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
-        const Item item = load_item(ws, it);
-        const int n = load_len(lengths, item.bh / H, L);
+      Item nxt = load_item_or_empty(ws, item_slot(0), count);
+
+      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
+        const Item item = nxt;
+        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+        const int n = item.n;
         const int row0 = item.blk * (C::BM * C::NQ);
         const int ntiles = (row0 + C::BM < n) ? 2 : 1;
         const int nkb = ceil_div(n, C::BN);
@@ -284,9 +292,11 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     constexpr float half_scale = 0.5f * Scale<D>::value;
     uint32_t sph = 0, oph = 0, turn_ph = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < count; it += gridDim.x) {
-      const Item item = load_item(ws, it);
-      const int n = load_len(lengths, item.bh / H, L);
+    Item nxt = load_item_or_empty(ws, item_slot(0), count);
+    for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
+      const Item item = nxt;
+      nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+      const int n = item.n;
       const bool two_tiles = item.blk * (C::BM * C::NQ) + C::BM < n;
       const int row0 = item.blk * (C::BM * C::NQ) + t * C::BM;
       const int row = row0 + r;
@@ -373,8 +383,8 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
 }
 
 template <int D>
-cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                            const int* lengths, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream) {
+cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
+                            int B, int H, int L, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D>;
   static bool configured[64] = {};
   int dev = 0;
@@ -386,15 +396,14 @@ cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const 
   }
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kFwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
-  fwd_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), lengths,
-                                                             ws, H, L);
-  return cudaGetLastError();
+  return launch_programmatic(fwd_kernel<D>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, tq, tk, tv,
+                             static_cast<__nv_bfloat16*>(o), ws, H, L);
 }
 
-cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                       const int* lengths, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream) {
-  if (d == 64) return launch_fwd_impl<64>(tq, tk, tv, o, lengths, ws, B, H, L, num_sms, stream);
-  return launch_fwd_impl<128>(tq, tk, tv, o, lengths, ws, B, H, L, num_sms, stream);
+cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
+                       int B, int H, int L, int num_sms, cudaStream_t stream) {
+  if (d == 64) return launch_fwd_impl<64>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+  return launch_fwd_impl<128>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
 }
 
 }  // namespace sigattn

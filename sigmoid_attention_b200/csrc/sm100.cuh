@@ -98,6 +98,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // ---------------------------------------------------------------------------
 // TMA (tensor-map tile loads into shared memory, completion on an mbarrier)
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. grid_dep_launch: this CTA allows the next
+// kernel in the stream (launched with programmatic stream serialization) to
+// start. grid_dep_wait: block until the previous kernel in the stream has
+// completed and its memory is visible (a no-op without a programmatic edge).
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

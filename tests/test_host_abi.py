@@ -36,9 +36,9 @@ def test_status_strings_and_sizes():
     assert "timed out" in sa.sigattn_status_str(4)
     assert [sa.sigattn_block_rows(k) for k in (0, 1, 2)] == [256, 128, 128]
     assert sa.sigattn_block_rows(3) == -1
-    # header + one 8-byte entry per possible 128-row item
-    assert sa.sigattn_workspace_size(4, 16, 4096, 128) == 256 + 8 * 4 * 16 * 32
-    assert sa.sigattn_workspace_size(2, 2, 64, 64) == 256 + 8 * 4
+    # header + one 16-byte entry per possible 128-row item
+    assert sa.sigattn_workspace_size(4, 16, 4096, 128) == 256 + 16 * 4 * 16 * 32
+    assert sa.sigattn_workspace_size(2, 2, 64, 64) == 256 + 16 * 4
     assert sa.sigattn_workspace_size(1, 1, 1, 96) == 0      # unsupported head size
     assert sa.sigattn_workspace_size(0, 1, 1, 64) == 0
     assert sa.sigattn_workspace_size(5000, 1, 1, 64) == 0   # beyond SIGATTN_MAX_BATCH
