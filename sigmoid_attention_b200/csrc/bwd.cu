@@ -87,6 +87,7 @@ struct BwdBarriers {
   uint64_t p_free, ds_free;        // the accumulation products of a block have read P / dS
   uint64_t acc_full, acc_empty;
   uint64_t drain[4];
+  ItemRing ring;
   uint32_t tmem_base;
   int abort;
 };
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     mbar_init(&bar.acc_full, KV ? 2 : 1);
     mbar_init(&bar.acc_empty, C::EPI_WARPS);
     for (int i = 0; i < 4; ++i) mbar_init(&bar.drain[i], 1);
+    ring_init(bar.ring, C::ISSUERS + C::EPI_WARPS);  // every issuer and epilogue warp reads each item
     bar.abort = 0;
     fence_mbar_init();
   }
@@ -170,10 +172,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       for (int s = 0; s < C::ST1; ++s) c1_last[s] = -1;
       for (int s = 0; s < C::ST2; ++s) c2_last[s] = -1;
       bool ok = true;
-      Item nxt = load_item_or_empty(ws, item_slot(0), count);
-      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
-        const Item item = nxt;
-        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+      uint32_t ist = 0, iph = 0;
+      int claimed = -1;
+      while (ok) {
+        const Item item = next_item(ws, claimed, count);
+        if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, ws, 200))) break;
+        if (item.n < 0) break;
         const int n = item.n;
         const int nb = ceil_div(n, C::BN);
         if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, ws, 201))) break;
@@ -185,6 +189,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         r_last = static_cast<int>(rph);
         rph ^= 1;
         for (int j = 0; j < nb; ++j) {
+          // Claim the CTA's next item two column blocks before this one ends.
+          if (j == max(0, nb - 2)) claimed = atomicAdd(ws + kHdrNext, 1);
           if (!(ok = mbar_wait(&bar.c1_empty[s1], p1 ^ 1, abort_flag, ws, 202))) break;
           mbar_arrive_expect_tx(&bar.c1_full[s1], C::TILE_C);
           for (int c = 0; c < D / 64; ++c)
@@ -225,10 +231,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       uint32_t st = 0, cph = 0, rph = 0, xb = 0;
       uint32_t read_ph[2] = {0, 0};
       bool ok = true;
-      Item nxt = load_item_or_empty(ws, item_slot(0), count);
-      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
-        const Item item = nxt;
-        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+      uint32_t ist = 0, iph = 0;
+      while (ok) {
+        Item item;
+        if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 210))) break;
+        ring_release(bar.ring, ist, iph, true);
+        if (item.n < 0) break;
         const int n = item.n;
         const int nb = ceil_div(n, C::BN);
         if (!(ok = mbar_wait(&bar.r_full, rph, abort_flag, ws, 211))) break;
@@ -279,10 +287,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       uint32_t st = 0, cph = 0, aph = 0;
       uint32_t fph[4] = {0, 0, 0, 0};
       bool ok = true;
-      Item nxt = load_item_or_empty(ws, item_slot(0), count);
-      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
-        const Item item = nxt;
-        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+      uint32_t ist = 0, iph = 0;
+      while (ok) {
+        Item item;
+        if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 210))) break;
+        ring_release(bar.ring, ist, iph, true);
+        if (item.n < 0) break;
         const int n = item.n;
         const int nb = ceil_div(n, C::BN);
         for (int j = 0; ok && j < nb; ++j) {
@@ -330,10 +340,13 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     uint32_t s_ph = 0, free_ph = 0, aph = 0, xb = 0;
     uint32_t dp_ph[2] = {0, 0};
     bool ok = true;
-    Item nxt = load_item_or_empty(ws, item_slot(0), count);
-    for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
-      const Item item = nxt;
-      nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+    uint32_t ist = 0, iph = 0;
+    while (ok) {
+      Item item;
+      if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 220))) break;
+      __syncwarp();
+      ring_release(bar.ring, ist, iph, lane == 0);
+      if (item.n < 0) break;
       const int n = item.n;
       const int nb = ceil_div(n, C::BN);
       const float half_bias = -0.5f * __logf(static_cast<float>(n));

@@ -53,20 +53,58 @@ __device__ __forceinline__ Item load_item(const int* ws, int idx) {
   return Item{v.x, v.y, v.z};
 }
 
-// Index of the item a persistent CTA takes in its round r. The plan lists the
-// items longest first; dealing them out in serpentine order (CTAs 0..G-1,
-// then G-1..0, ...) evens out the per-CTA totals better than plain
-// round-robin, which gives CTA 0 the longest item of every round. Increases
-// with r, so a CTA is done at its first index >= count.
-__device__ __forceinline__ int item_slot(int r) {
-  const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
-  return r * g + ((r & 1) ? g - 1 - b : b);
+constexpr Item kNoItem{0, 0, -1};  // end of the work list
+
+// Dynamic longest-processing-time-first scheduling. The plan lists the items
+// longest first; each CTA's producer takes item blockIdx.x first and every
+// later one from the claim counter in the workspace header, so a CTA gets the
+// next item of the list when it is ready for one. The producer hands each
+// item to the CTA's other roles through this two-slot ring in shared memory
+// (so they never wait on a global load for it); after the last item it
+// publishes kNoItem.
+struct ItemRing {
+  int4 slot[2];
+  uint64_t full[2];   // count 1: the producer wrote the slot
+  uint64_t empty[2];  // count = consumer arrivals per item
+};
+
+__device__ __forceinline__ void ring_init(ItemRing& r, int consumers) {
+  for (int s = 0; s < 2; ++s) {
+    mbar_init(&r.full[s], 1);
+    mbar_init(&r.empty[s], consumers);
+  }
 }
 
-// The item at `idx` (or an empty one past the end).
-// Loaded one item ahead, so the load's latency is off the item boundary.
-__device__ __forceinline__ Item load_item_or_empty(const int* ws, int idx, int count) {
-  return idx < count ? load_item(ws, idx) : Item{0, 0, 0};
+// Producer: the CTA's next item (its first is `blockIdx.x`, `claimed` holds a
+// counter value taken earlier, or -1 for the first call).
+__device__ __forceinline__ Item next_item(const int* ws, int claimed, int count) {
+  const int idx = claimed < 0 ? static_cast<int>(blockIdx.x) : claimed + static_cast<int>(gridDim.x);
+  return idx < count ? load_item(ws, idx) : kNoItem;
+}
+
+__device__ __forceinline__ bool ring_publish(ItemRing& r, uint32_t& st, uint32_t& ph, const Item& item,
+                                             volatile int* abort_flag, int* ws, int site) {
+  if (!mbar_wait(&r.empty[st], ph ^ 1, abort_flag, ws, site)) return false;
+  r.slot[st] = make_int4(item.bh, item.blk, item.n, 0);
+  mbar_arrive(&r.full[st]);
+  if (++st == 2) { st = 0; ph ^= 1; }
+  return true;
+}
+
+// Consumer side: wait for the next slot and copy the item out. A single
+// consuming thread releases the slot with ring_release at once; a warp
+// releases it once every lane has read it (__syncwarp, then lane 0).
+__device__ __forceinline__ bool ring_read(ItemRing& r, uint32_t st, uint32_t ph, Item* item,
+                                          volatile int* abort_flag, int* ws, int site) {
+  if (!mbar_wait(&r.full[st], ph, abort_flag, ws, site)) return false;
+  const int4 v = r.slot[st];  // ordered after the wait by its acquire and memory clobber
+  *item = Item{v.x, v.y, v.z};
+  return true;
+}
+
+__device__ __forceinline__ void ring_release(ItemRing& r, uint32_t& st, uint32_t& ph, bool arrive) {
+  if (arrive) mbar_arrive(&r.empty[st]);
+  if (++st == 2) { st = 0; ph ^= 1; }
 }
 
 // 1/sqrt(d) for the supported head sizes.

@@ -62,6 +62,7 @@ struct FwdBarriers {
   uint64_t s_full[2], p_full[4], o_full[2], o_empty[2];
   uint64_t epi_done[2];  // tile t's warps finished their sigmoid pass over a block
   uint64_t drain[2];
+  ItemRing ring;
   uint32_t tmem_base;
   int abort;
 };
@@ -101,6 +102,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     mbar_init(&bar.epi_done[1], 8);
     mbar_init(&bar.drain[0], 1);
     mbar_init(&bar.drain[1], 1);
+    ring_init(bar.ring, 2 + C::EPI_WARPS);  // both issuers and every epilogue warp read each item
     bar.abort = 0;
     fence_mbar_init();
   }
@@ -130,10 +132,12 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       for (int s = 0; s < C::KST; ++s) k_last[s] = -1;
       for (int s = 0; s < C::VST; ++s) v_last[s] = -1;
       bool ok = true;
-      Item nxt = load_item_or_empty(ws, item_slot(0), count);
-      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
-        const Item item = nxt;
-        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+      uint32_t ist = 0, iph = 0;
+      int claimed = -1;
+      while (ok) {
+        const Item item = next_item(ws, claimed, count);
+        if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, ws, 100))) break;
+        if (item.n < 0) break;
         const int n = item.n;
         const int row0 = item.blk * (C::BM * C::NQ);
         const int ntiles = (row0 + C::BM < n) ? 2 : 1;
@@ -147,6 +151,8 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
         q_last = static_cast<int>(qph);
         qph ^= 1;
         for (int j = 0; j < nkb; ++j) {
+          // Claim the CTA's next item two key blocks before this one ends.
+          if (j == max(0, nkb - 2)) claimed = atomicAdd(ws + kHdrNext, 1);
           if (!(ok = mbar_wait(&bar.k_empty[kst], kph ^ 1, abort_flag, ws, 102))) break;
           mbar_arrive_expect_tx(&bar.k_full[kst], C::TILE_BYTES);
           for (int c = 0; c < D / 64; ++c)
@@ -211,11 +217,12 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       auto advance_k = [&]() { if (++kst == C::KST) { kst = 0; kph ^= 1; } };
       auto advance_v = [&]() { if (++vst == C::VST) { vst = 0; vph ^= 1; } };
 
-      Item nxt = load_item_or_empty(ws, item_slot(0), count);
-
-      for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
-        const Item item = nxt;
-        nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+      uint32_t ist = 0, iph = 0;
+      while (ok) {
+        Item item;
+        if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 110))) break;
+        ring_release(bar.ring, ist, iph, true);
+        if (item.n < 0) break;
         const int n = item.n;
         const int row0 = item.blk * (C::BM * C::NQ);
         const int ntiles = (row0 + C::BM < n) ? 2 : 1;
@@ -292,10 +299,13 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     constexpr float half_scale = 0.5f * Scale<D>::value;
     uint32_t sph = 0, oph = 0, turn_ph = 0;
     bool ok = true;
-    Item nxt = load_item_or_empty(ws, item_slot(0), count);
-    for (int rnd = 0; ok && item_slot(rnd) < count; ++rnd) {
-      const Item item = nxt;
-      nxt = load_item_or_empty(ws, item_slot(rnd + 1), count);
+    uint32_t ist = 0, iph = 0;
+    while (ok) {
+      Item item;
+      if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 120))) break;
+      __syncwarp();
+      ring_release(bar.ring, ist, iph, lane == 0);
+      if (item.n < 0) break;
       const int n = item.n;
       const bool two_tiles = item.blk * (C::BM * C::NQ) + C::BM < n;
       const int row0 = item.blk * (C::BM * C::NQ) + t * C::BM;

@@ -76,7 +76,10 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
   }
   __syncthreads();
   const int total = s_off[B];
-  if (tid == 0) ws[kHdrCount] = total;
+  if (tid == 0) {
+    ws[kHdrCount] = total;
+    ws[kHdrNext] = 0;  // the compute kernel's claim counter
+  }
   int4* items = reinterpret_cast<int4*>(ws + kHeaderWords);
   for (int i = tid; i < total; i += blockDim.x) {
     int lo = 0, hi = B - 1;  // find s with s_off[s] <= i < s_off[s + 1]

@@ -23,6 +23,7 @@ enum : int {
   kHdrError = 0,      // sticky: 0 = fine, else a sigattn_status code
   kHdrErrorSite = 1,  // which wait timed out / which check failed
   kHdrCount = 2,      // number of work items in the list
+  kHdrNext = 3,       // work-item claim counter of the compute kernels (zeroed by the plan)
   kHeaderWords = 64,  // 256 bytes
 };
 
