@@ -103,6 +103,35 @@ SIGATTN_API int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, co
                      const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* Packed ("varlen") layout: the same three operations on sequences stored
+ * back to back instead of padded to Lmax, so padding costs neither FLOPs nor
+ * HBM bytes. Sequence b's tokens are rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+ * of every tensor; n_b = cu_seqlens[b+1] - cu_seqlens[b].
+ *  - Tensors are bf16, contiguous [total][H][d] (d fastest, then heads, then
+ *    tokens), in device memory, 16-byte aligned; d is 64 or 128.
+ *  - cu_seqlens is int32 [B+1] in device memory, nondecreasing, with
+ *    0 <= cu_seqlens[b] and cu_seqlens[B] <= total. max_seqlen >= every n_b
+ *    plays the part of Lmax (work-list size, limits). A sequence whose bounds
+ *    break these rules gets no work: its rows are left untouched and
+ *    SIGATTN_ERR_INVALID_ARG is raised in the workspace's sticky error word.
+ *  - Only rows that belong to a sequence are written; rows outside every
+ *    [cu_seqlens[b], cu_seqlens[b+1]) are never touched. Results equal those of
+ *    the padded calls on the same sequences. The last row block of a sequence
+ *    reads up to 255 rows past its end (the next sequence, or rows after
+ *    cu_seqlens[B]); those enter only as 0 * value and must be finite, as
+ *    padded rows must be in the padded layout.
+ *  - 1 <= total <= INT32_MAX - 4096; workspace: sigattn_workspace_size(B, H,
+ *    max_seqlen, d) bytes. Everything else as for the padded calls. */
+SIGATTN_API int sigattn_fwd_varlen(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
+                                   int B, int H, int max_seqlen, int total, int d, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+SIGATTN_API int sigattn_bwd_dq_varlen(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                                      const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total, int d,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+SIGATTN_API int sigattn_bwd_dkdv_varlen(const void* q, const void* k, const void* v, const void* dout, void* dk,
+                                        void* dv, const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total,
+                                        int d, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Run only the ragged tile scheduler for `kind` on the device: afterwards the
  * workspace holds, at byte offset 8, the item count (int32), and at byte
  * offset 256, `count` entries of four int32 (bh = b*H + h, block index, the

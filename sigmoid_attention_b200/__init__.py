@@ -22,6 +22,7 @@ __all__ = [
     "SigattnError", "library", "library_path", "sigattn_version", "sigattn_status_str", "sigattn_block_rows",
     "sigattn_workspace_size", "sigattn_fwd", "sigattn_fwd_noalloc", "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
     "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
+    "sigattn_fwd_varlen", "sigattn_bwd_dq_varlen", "sigattn_bwd_dkdv_varlen",
     "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
 ]
 
@@ -69,6 +70,12 @@ def library():
         lib.sigattn_bwd_dq.argtypes = [_vp] * 6 + [_i] * 4 + [_vp, _sz, _vp]
         lib.sigattn_bwd_dkdv.restype = _i
         lib.sigattn_bwd_dkdv.argtypes = [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]
+        lib.sigattn_fwd_varlen.restype = _i
+        lib.sigattn_fwd_varlen.argtypes = [_vp] * 5 + [_i] * 5 + [_vp, _sz, _vp]
+        lib.sigattn_bwd_dq_varlen.restype = _i
+        lib.sigattn_bwd_dq_varlen.argtypes = [_vp] * 6 + [_i] * 5 + [_vp, _sz, _vp]
+        lib.sigattn_bwd_dkdv_varlen.restype = _i
+        lib.sigattn_bwd_dkdv_varlen.argtypes = [_vp] * 7 + [_i] * 5 + [_vp, _sz, _vp]
         lib.sigattn_plan.restype = _i
         lib.sigattn_plan.argtypes = [_vp] + [_i] * 5 + [_vp, _sz, _vp]
         lib.sigattn_plan_host.restype = _i
@@ -166,6 +173,40 @@ def sigattn_bwd_dkdv(q, k, v, dout, dk, dv, lengths, workspace, stream=None) -> 
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dk, "dk"), _dev(dv, "dv"),
         _dev(lengths, "lengths", torch.int32), B, H, L, d, _dev(workspace, "workspace", torch.uint8),
         workspace.numel(), _stream_ptr(stream)))
+
+
+def _packed_dims(q: torch.Tensor):
+    if q.dim() != 3:
+        raise ValueError("expected a packed [total, H, d] tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def sigattn_fwd_varlen(q, k, v, o, cu_seqlens, max_seqlen: int, workspace, stream=None) -> None:
+    """Packed layout: q, k, v, o are [total, H, d]; cu_seqlens is int32 [B + 1]."""
+    total, H, d = _packed_dims(q)
+    B = cu_seqlens.numel() - 1
+    _check("sigattn_fwd_varlen", library().sigattn_fwd_varlen(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(cu_seqlens, "cu_seqlens", torch.int32),
+        B, H, int(max_seqlen), total, d, _dev(workspace, "workspace", torch.uint8), workspace.numel(),
+        _stream_ptr(stream)))
+
+
+def sigattn_bwd_dq_varlen(q, k, v, dout, dq, cu_seqlens, max_seqlen: int, workspace, stream=None) -> None:
+    total, H, d = _packed_dims(q)
+    B = cu_seqlens.numel() - 1
+    _check("sigattn_bwd_dq_varlen", library().sigattn_bwd_dq_varlen(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dq, "dq"),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), B, H, int(max_seqlen), total, d,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_bwd_dkdv_varlen(q, k, v, dout, dk, dv, cu_seqlens, max_seqlen: int, workspace, stream=None) -> None:
+    total, H, d = _packed_dims(q)
+    B = cu_seqlens.numel() - 1
+    _check("sigattn_bwd_dkdv_varlen", library().sigattn_bwd_dkdv_varlen(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dk, "dk"), _dev(dv, "dv"),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), B, H, int(max_seqlen), total, d,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
 
 
 def sigattn_plan(lengths, B, H, Lmax, d, kind, workspace, stream=None) -> None:

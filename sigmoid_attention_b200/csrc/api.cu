@@ -10,17 +10,18 @@
 #include "common.cuh"
 
 namespace sigattn {
-cudaError_t launch_prep(const int* lengths, int B, int H, int L, int kind, int* ws, cudaStream_t stream);
+cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, int* ws,
+                        cudaStream_t stream);
 cudaError_t launch_fill(const int* lengths, int B, int H, int L, int d, int kind, void* out0, void* out1,
                         int num_sms, cudaStream_t stream);
 int plan_host(const int* lengths, int B, int H, int L, int kind, int* out, int cap);
 cudaError_t launch_selftest_timeout(int* ws, unsigned long long limit_ns, cudaStream_t stream);
-cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
-                       int B, int H, int L, int num_sms, cudaStream_t stream);
-cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+cudaError_t launch_fwd(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       void* o, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_dq(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                           const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L, int num_sms,
                           cudaStream_t stream);
-cudaError_t launch_bwd_dkdv(int d, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+cudaError_t launch_bwd_dkdv(int d, bool packed, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                             const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int L, int num_sms,
                             cudaStream_t stream);
 void set_last_error(const char* msg);
@@ -93,6 +94,26 @@ bool make_map(CUtensorMap* map, const void* ptr, int BH, int L, int d, int box_r
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// 3-D view {d, H, total} of a packed [total][H][d] bf16 tensor, loaded as
+// [box_rows tokens][1 head][64 columns] boxes (the same shared-memory image as
+// a [box_rows][64] box). Tokens past `total` read as zeros.
+bool make_map_packed(CUtensorMap* map, const void* ptr, int total, int H, int d, int box_rows = 128) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, elem,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed token count bound: token coordinates start_b + row (row < n_b + 256)
+// stay in int32.
+constexpr int kMaxPackedTokens = INT_MAX - 4096;
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -181,8 +202,8 @@ int sigattn_fwd(const void* q, const void* k, const void* v, void* o, const int3
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, B, H, Lmax, SIGATTN_KIND_FWD, ws, s));
-  if (st == SIGATTN_OK) st = cuda_status(launch_fwd(d, tq, tk, tv, o, ws, B, H, Lmax, info.num_sms, s));
+  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_FWD, ws, s));
+  if (st == SIGATTN_OK) st = cuda_status(launch_fwd(d, false, tq, tk, tv, o, ws, B, H, Lmax, info.num_sms, s));
   if (st != SIGATTN_OK) return st;
   return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_FWD, o, nullptr, info.num_sms, s));
 }
@@ -200,8 +221,9 @@ int sigattn_bwd_dq(const void* q, const void* k, const void* v, const void* dout
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, B, H, Lmax, SIGATTN_KIND_DQ, ws, s));
-  if (st == SIGATTN_OK) st = cuda_status(launch_bwd_dq(d, tq, tdo, tk, tv, dq, ws, B, H, Lmax, info.num_sms, s));
+  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_DQ, ws, s));
+  if (st == SIGATTN_OK)
+    st = cuda_status(launch_bwd_dq(d, false, tq, tdo, tk, tv, dq, ws, B, H, Lmax, info.num_sms, s));
   if (st != SIGATTN_OK) return st;
   return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_DQ, dq, nullptr, info.num_sms, s));
 }
@@ -223,11 +245,71 @@ int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* do
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, B, H, Lmax, SIGATTN_KIND_DKDV, ws, s));
+  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_DKDV, ws, s));
   if (st == SIGATTN_OK)
-    st = cuda_status(launch_bwd_dkdv(d, tk, tv, tq, tdo, dk, dv, ws, B, H, Lmax, info.num_sms, s));
+    st = cuda_status(launch_bwd_dkdv(d, false, tk, tv, tq, tdo, dk, dv, ws, B, H, Lmax, info.num_sms, s));
   if (st != SIGATTN_OK) return st;
   return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_DKDV, dk, dv, info.num_sms, s));
+}
+
+int sigattn_fwd_varlen(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens, int B,
+                       int H, int max_seqlen, int total, int d, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, max_seqlen, d, cu_seqlens, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (total < 1 || total > kMaxPackedTokens) return total < 1 ? SIGATTN_ERR_INVALID_ARG : SIGATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SIGATTN_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  if (!make_map_packed(&tq, q, total, H, d) || !make_map_packed(&tk, k, total, H, d) ||
+      !make_map_packed(&tv, v, total, H, d))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_FWD, ws, s));
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(launch_fwd(d, true, tq, tk, tv, o, ws, B, H, max_seqlen, info.num_sms, s));
+}
+
+int sigattn_bwd_dq_varlen(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                          const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total, int d, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, max_seqlen, d, cu_seqlens, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (total < 1 || total > kMaxPackedTokens) return total < 1 ? SIGATTN_ERR_INVALID_ARG : SIGATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq))
+    return SIGATTN_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map_packed(&tq, q, total, H, d) || !make_map_packed(&tk, k, total, H, d) ||
+      !make_map_packed(&tv, v, total, H, d) || !make_map_packed(&tdo, dout, total, H, d))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_DQ, ws, s));
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(launch_bwd_dq(d, true, tq, tdo, tk, tv, dq, ws, B, H, max_seqlen, info.num_sms, s));
+}
+
+int sigattn_bwd_dkdv_varlen(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                            const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total, int d,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, max_seqlen, d, cu_seqlens, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (total < 1 || total > kMaxPackedTokens) return total < 1 ? SIGATTN_ERR_INVALID_ARG : SIGATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
+    return SIGATTN_ERR_INVALID_ARG;
+  const int cb = bwd_col_block(true, d);
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map_packed(&tq, q, total, H, d, cb) || !make_map_packed(&tk, k, total, H, d) ||
+      !make_map_packed(&tv, v, total, H, d) || !make_map_packed(&tdo, dout, total, H, d, cb))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_DKDV, ws, s));
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(launch_bwd_dkdv(d, true, tk, tv, tq, tdo, dk, dv, ws, B, H, max_seqlen, info.num_sms, s));
 }
 
 int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind, void* workspace,
@@ -236,8 +318,8 @@ int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind
   DeviceInfo info;
   int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
   if (st != SIGATTN_OK) return st;
-  return cuda_status(
-      launch_prep(lengths, B, H, Lmax, kind, static_cast<int*>(workspace), static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, kind, static_cast<int*>(workspace),
+                                 static_cast<cudaStream_t>(stream)));
 }
 
 int sigattn_plan_host(const int32_t* lengths_host, int B, int H, int Lmax, int kind, int32_t* items_out, int cap,

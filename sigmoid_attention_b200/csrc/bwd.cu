@@ -92,7 +92,7 @@ struct BwdBarriers {
   int abort;
 };
 
-template <int D, bool KV>
+template <int D, bool KV, bool PACKED>
 __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_r1, const __grid_constant__ CUtensorMap tm_r2,
                const __grid_constant__ CUtensorMap tm_c1, const __grid_constant__ CUtensorMap tm_c2,
@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
   const int count = ws[kHdrCount];
+  const RowMap<PACKED> rm{H, L};
 
   // Descriptor bases (built once, advanced by adding (bytes >> 4): the
   // start-address field is the low 14 bits and smem stays below 256 KB).
@@ -179,12 +180,14 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, ws, 200))) break;
         if (item.n < 0) break;
         const int n = item.n;
+        const int hd = PACKED ? item.bh % H : 0;
         const int nb = ceil_div(n, C::BN);
         if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, ws, 201))) break;
         mbar_arrive_expect_tx(&bar.r_full, 2 * C::TILE_R);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem + C::OFF_R1 + c * C::BOX_R, &tm_r1, &bar.r_full, c * 64, item.blk * C::BM, item.bh);
-          tma_load_3d(smem + C::OFF_R2 + c * C::BOX_R, &tm_r2, &bar.r_full, c * 64, item.blk * C::BM, item.bh);
+          const int ry = rm.y(item, hd, item.blk * C::BM), rz = rm.z(item, item.blk * C::BM);
+          tma_load_3d(smem + C::OFF_R1 + c * C::BOX_R, &tm_r1, &bar.r_full, c * 64, ry, rz);
+          tma_load_3d(smem + C::OFF_R2 + c * C::BOX_R, &tm_r2, &bar.r_full, c * 64, ry, rz);
         }
         r_last = static_cast<int>(rph);
         rph ^= 1;
@@ -195,14 +198,14 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           mbar_arrive_expect_tx(&bar.c1_full[s1], C::TILE_C);
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(smem + C::OFF_C1 + s1 * C::TILE_C + c * C::BOX_C, &tm_c1, &bar.c1_full[s1], c * 64,
-                        j * C::BN, item.bh);
+                        rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
           c1_last[s1] = static_cast<int>(p1);
           if (++s1 == C::ST1) { s1 = 0; p1 ^= 1; }
           if (!(ok = mbar_wait(&bar.c2_empty[s2], p2 ^ 1, abort_flag, ws, 203))) break;
           mbar_arrive_expect_tx(&bar.c2_full[s2], C::TILE_C);
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(smem + C::OFF_C2 + s2 * C::TILE_C + c * C::BOX_C, &tm_c2, &bar.c2_full[s2], c * 64,
-                        j * C::BN, item.bh);
+                        rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
           c2_last[s2] = static_cast<int>(p2);
           if (++s2 == C::ST2) { s2 = 0; p2 ^= 1; }
         }
@@ -442,9 +445,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       aph ^= 1;
       tc_fence_after();
       const int row = item.blk * C::BM + r;
-      const bool in_range = row < L;
+      const bool in_range = rm.writes(row, n);
       const bool valid_row = row < n;
-      const size_t row_off = (static_cast<size_t>(item.bh) * L + row) * D;
+      const size_t row_off = rm.offset(item, PACKED ? item.bh % H : 0, row, D);
       // 32-column chunks of the accumulators: A1 (-> out1, times scale), then
       // A2 (-> out2) for dK/dV; each half of the warps takes every other
       // chunk. Each chunk is copied out and packed to bf16 at once, so the
@@ -495,7 +498,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   }
 }
 
-template <int D, bool KV>
+template <int D, bool KV, bool PACKED>
 cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
                             const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
                             cudaStream_t stream) {
@@ -505,28 +508,38 @@ cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const 
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(bwd_kernel<D, KV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+        cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kBwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
-  return launch_programmatic(bwd_kernel<D, KV>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2, c1, c2,
-                             static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), ws, H, L);
+  return launch_programmatic(bwd_kernel<D, KV, PACKED>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2,
+                             c1, c2, static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), ws, H, L);
 }
 
-cudaError_t launch_bwd_dq(int d, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+template <bool KV>
+cudaError_t launch_bwd(int d, bool packed, const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
+                       const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
+                       cudaStream_t stream) {
+  if (packed) {
+    if (d == 64) return launch_bwd_impl<64, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, stream);
+    return launch_bwd_impl<128, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, stream);
+  }
+  if (d == 64) return launch_bwd_impl<64, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, stream);
+  return launch_bwd_impl<128, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, stream);
+}
+
+cudaError_t launch_bwd_dq(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                           const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L, int num_sms,
                           cudaStream_t stream) {
-  if (d == 64) return launch_bwd_impl<64, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, num_sms, stream);
-  return launch_bwd_impl<128, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, num_sms, stream);
+  return launch_bwd<false>(d, packed, tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, num_sms, stream);
 }
 
-cudaError_t launch_bwd_dkdv(int d, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+cudaError_t launch_bwd_dkdv(int d, bool packed, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                             const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int L, int num_sms,
                             cudaStream_t stream) {
-  if (d == 64) return launch_bwd_impl<64, true>(tk, tv, tq, tdo, dk, dv, ws, B, H, L, num_sms, stream);
-  return launch_bwd_impl<128, true>(tk, tv, tq, tdo, dk, dv, ws, B, H, L, num_sms, stream);
+  return launch_bwd<true>(d, packed, tk, tv, tq, tdo, dk, dv, ws, B, H, L, num_sms, stream);
 }
 
 }  // namespace sigattn

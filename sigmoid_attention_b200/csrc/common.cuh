@@ -40,20 +40,41 @@ __device__ __forceinline__ int load_len(const int* lengths, int b, int L) {
   return (n < 0 || n > L) ? 0 : n;
 }
 
-// One work item as the plan stores it: 16 bytes {b * H + h, row block, n_b, 0},
-// so a kernel learns the item and its sequence's valid length from one load.
+// One work item as the plan stores it: 16 bytes {b * H + h, row block, n_b,
+// start_b}, so a kernel learns the item, its sequence's valid length and (for
+// packed inputs) the sequence's first token from one load.
 struct Item {
-  int bh;   // b * H + h
-  int blk;  // row-block index within the slice
-  int n;    // valid length of sequence b
+  int bh;     // b * H + h
+  int blk;    // row-block index within the slice
+  int n;      // valid length of sequence b
+  int start;  // packed layout: index of the sequence's first token (0 when padded)
 };
 
 __device__ __forceinline__ Item load_item(const int* ws, int idx) {
   const int4 v = reinterpret_cast<const int4*>(ws + kHeaderWords)[idx];
-  return Item{v.x, v.y, v.z};
+  return Item{v.x, v.y, v.z, v.w};
 }
 
-constexpr Item kNoItem{0, 0, -1};  // end of the work list
+// Where the rows of a (b, h) slice live, for both input layouts.
+//  padded [B][H][Lmax][d]: TMA view {d, Lmax, B*H}; row r of slice bh is at
+//    (y, z) = (r, bh). Rows n_b <= r < Lmax are padding and are written as zeros.
+//  packed [total][H][d] (sequence b holds tokens start_b .. start_b + n_b - 1):
+//    TMA view {d, H, total}; row r is at (y, z) = (h, start_b + r). Rows r >= n_b
+//    belong to the next sequence and are never written.
+template <bool PACKED>
+struct RowMap {
+  int H, L;
+  __device__ __forceinline__ int y(const Item& it, int h, int row) const { return PACKED ? h : row; }
+  __device__ __forceinline__ int z(const Item& it, int row) const { return PACKED ? it.start + row : it.bh; }
+  // Element offset of the row in an output tensor of head size D.
+  __device__ __forceinline__ size_t offset(const Item& it, int h, int row, int D) const {
+    return PACKED ? (static_cast<size_t>(it.start + row) * H + h) * D : (static_cast<size_t>(it.bh) * L + row) * D;
+  }
+  // Whether the item's epilogue writes this row (zeros when row >= n).
+  __device__ __forceinline__ bool writes(int row, int n) const { return PACKED ? row < n : row < L; }
+};
+
+constexpr Item kNoItem{0, 0, -1, 0};  // end of the work list
 
 // Dynamic longest-processing-time-first scheduling. The plan lists the items
 // longest first; each CTA's producer takes item blockIdx.x first and every
@@ -85,7 +106,7 @@ __device__ __forceinline__ Item next_item(const int* ws, int claimed, int count)
 __device__ __forceinline__ bool ring_publish(ItemRing& r, uint32_t& st, uint32_t& ph, const Item& item,
                                              volatile int* abort_flag, int* ws, int site) {
   if (!mbar_wait(&r.empty[st], ph ^ 1, abort_flag, ws, site)) return false;
-  r.slot[st] = make_int4(item.bh, item.blk, item.n, 0);
+  r.slot[st] = make_int4(item.bh, item.blk, item.n, item.start);
   mbar_arrive(&r.full[st]);
   if (++st == 2) { st = 0; ph ^= 1; }
   return true;
@@ -98,7 +119,7 @@ __device__ __forceinline__ bool ring_read(ItemRing& r, uint32_t st, uint32_t ph,
                                           volatile int* abort_flag, int* ws, int site) {
   if (!mbar_wait(&r.full[st], ph, abort_flag, ws, site)) return false;
   const int4 v = r.slot[st];  // ordered after the wait by its acquire and memory clobber
-  *item = Item{v.x, v.y, v.z};
+  *item = Item{v.x, v.y, v.z, v.w};
   return true;
 }
 

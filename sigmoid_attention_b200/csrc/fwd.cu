@@ -67,7 +67,7 @@ struct FwdBarriers {
   int abort;
 };
 
-template <int D>
+template <int D, bool PACKED>
 __global__ void __launch_bounds__((16 + 3) * 32, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
@@ -118,6 +118,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
   const int count = ws[kHdrCount];
+  const RowMap<PACKED> rm{H, L};
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------- producer
@@ -139,6 +140,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
         if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, ws, 100))) break;
         if (item.n < 0) break;
         const int n = item.n;
+        const int hd = PACKED ? item.bh % H : 0;
         const int row0 = item.blk * (C::BM * C::NQ);
         const int ntiles = (row0 + C::BM < n) ? 2 : 1;
         const int nkb = ceil_div(n, C::BN);
@@ -146,8 +148,8 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
         mbar_arrive_expect_tx(&bar.q_full, ntiles * C::TILE_BYTES);
         for (int t = 0; t < ntiles; ++t)
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ + t * C::TILE_BYTES + c * C::BOX_BYTES, &tm_q, &bar.q_full, c * 64, row0 + t * C::BM,
-                        item.bh);
+            tma_load_3d(sQ + t * C::TILE_BYTES + c * C::BOX_BYTES, &tm_q, &bar.q_full, c * 64,
+                        rm.y(item, hd, row0 + t * C::BM), rm.z(item, row0 + t * C::BM));
         q_last = static_cast<int>(qph);
         qph ^= 1;
         for (int j = 0; j < nkb; ++j) {
@@ -156,15 +158,15 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           if (!(ok = mbar_wait(&bar.k_empty[kst], kph ^ 1, abort_flag, ws, 102))) break;
           mbar_arrive_expect_tx(&bar.k_full[kst], C::TILE_BYTES);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sK + kst * C::TILE_BYTES + c * C::BOX_BYTES, &tm_k, &bar.k_full[kst], c * 64, j * C::BN,
-                        item.bh);
+            tma_load_3d(sK + kst * C::TILE_BYTES + c * C::BOX_BYTES, &tm_k, &bar.k_full[kst], c * 64,
+                        rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
           k_last[kst] = static_cast<int>(kph);
           if (++kst == C::KST) { kst = 0; kph ^= 1; }
           if (!(ok = mbar_wait(&bar.v_empty[vst], vph ^ 1, abort_flag, ws, 103))) break;
           mbar_arrive_expect_tx(&bar.v_full[vst], C::TILE_BYTES);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sV + vst * C::TILE_BYTES + c * C::BOX_BYTES, &tm_v, &bar.v_full[vst], c * 64, j * C::BN,
-                        item.bh);
+            tma_load_3d(sV + vst * C::TILE_BYTES + c * C::BOX_BYTES, &tm_v, &bar.v_full[vst], c * 64,
+                        rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
           v_last[vst] = static_cast<int>(vph);
           if (++vst == C::VST) { vst = 0; vph ^= 1; }
         }
@@ -310,9 +312,9 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       const bool two_tiles = item.blk * (C::BM * C::NQ) + C::BM < n;
       const int row0 = item.blk * (C::BM * C::NQ) + t * C::BM;
       const int row = row0 + r;
-      __nv_bfloat16* orow = out + (static_cast<size_t>(item.bh) * L + row) * D + h * (D / 2);
-      if (row0 >= n) {  // tile fully padded: its rows of O are zero
-        if (row < L) {
+      __nv_bfloat16* orow = out + rm.offset(item, PACKED ? item.bh % H : 0, row, D) + h * (D / 2);
+      if (row0 >= n) {  // tile fully padded: its rows of O are zero (padded layout)
+        if (rm.writes(row, n)) {
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) store_zero32(orow + c * 32);
         }
@@ -374,7 +376,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.o_empty[t]);
-      if (row < L) {
+      if (rm.writes(row, n)) {
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           if (row < n) store_row32(orow + c * 32, v[c], 1.0f);
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
   }
 }
 
-template <int D>
+template <int D, bool PACKED>
 cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
                             int B, int H, int L, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D>;
@@ -400,20 +402,26 @@ cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const 
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+    cudaError_t e =
+        cudaFuncSetAttribute(fwd_kernel<D, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kFwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
-  return launch_programmatic(fwd_kernel<D>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, tq, tk, tv,
+  return launch_programmatic(fwd_kernel<D, PACKED>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, tq, tk, tv,
                              static_cast<__nv_bfloat16*>(o), ws, H, L);
 }
 
-cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
-                       int B, int H, int L, int num_sms, cudaStream_t stream) {
-  if (d == 64) return launch_fwd_impl<64>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
-  return launch_fwd_impl<128>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+// L is Lmax for the padded layout and the longest sequence for the packed one.
+cudaError_t launch_fwd(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       void* o, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream) {
+  if (packed) {
+    if (d == 64) return launch_fwd_impl<64, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+    return launch_fwd_impl<128, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+  }
+  if (d == 64) return launch_fwd_impl<64, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+  return launch_fwd_impl<128, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
 }
 
 }  // namespace sigattn

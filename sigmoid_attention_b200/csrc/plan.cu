@@ -25,8 +25,13 @@
 
 namespace sigattn {
 
-__global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ lengths, int B, int H, int L,
-                                                    int rows, int* __restrict__ ws) {
+// Sequence lengths come either from `lengths` (padded layout) or, when `cu`
+// is given, from cumulative offsets: sequence b holds packed tokens
+// [cu[b], cu[b+1]), which must lie inside [0, total_tokens]. A sequence that breaks
+// its bounds gets no work items and raises SIGATTN_ERR_INVALID_ARG.
+__global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ lengths, const int* __restrict__ cu,
+                                                    int total_tokens, int B, int H, int L, int rows,
+                                                    int* __restrict__ ws) {
   // The compute kernel that follows may set itself up meanwhile; it waits
   // for this grid before it reads the plan.
   grid_dep_launch();
@@ -35,13 +40,25 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
   int* s_len = smem_plan;            // [B]
   int* s_order = smem_plan + B;      // [B]
   int* s_off = smem_plan + 2 * B;    // [B + 1]
+  int* s_start = smem_plan + 3 * B + 1;  // [B]
   for (int b = tid; b < B; b += blockDim.x) {
-    const int n = __ldg(lengths + b);
-    if (n < 0 || n > L) {
+    int n, start = 0;
+    bool bad;
+    if (cu != nullptr) {
+      start = __ldg(cu + b);
+      const int end = __ldg(cu + b + 1);
+      n = end - start;
+      bad = start < 0 || end < start || end > total_tokens || n > L;
+    } else {
+      n = __ldg(lengths + b);
+      bad = n < 0 || n > L;
+    }
+    if (bad) {
       atomicCAS(ws + kHdrError, 0, 1 /* SIGATTN_ERR_INVALID_ARG */);
       atomicExch(ws + kHdrErrorSite, -(b + 1));
     }
-    s_len[b] = (n < 0 || n > L) ? 0 : n;
+    s_len[b] = bad ? 0 : n;
+    s_start[b] = bad ? 0 : start;
   }
   __syncthreads();
   // Rank of each sequence in the longest-first order (ties keep batch order).
@@ -90,23 +107,24 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
     const int b = s_order[lo];
     const int local = i - s_off[lo];
     const int nblk = ceil_div(s_len[b], rows);
-    items[i] = make_int4(b * H + local / nblk, local % nblk, s_len[b], 0);
+    items[i] = make_int4(b * H + local / nblk, local % nblk, s_len[b], s_start[b]);
   }
 }
 
-cudaError_t launch_prep(const int* lengths, int B, int H, int L, int kind, int* ws, cudaStream_t stream) {
-  const int smem = (3 * B + 1) * static_cast<int>(sizeof(int));
+cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, int* ws,
+                        cudaStream_t stream) {
+  const int smem = (4 * B + 1) * static_cast<int>(sizeof(int));
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (3 * kMaxBatch + 1) * static_cast<int>(sizeof(int)));
+                                         (4 * kMaxBatch + 1) * static_cast<int>(sizeof(int)));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int threads = B <= 256 ? 256 : 1024;
-  prep_kernel<<<1, threads, smem, stream>>>(lengths, B, H, L, item_rows(kind), ws);
+  prep_kernel<<<1, threads, smem, stream>>>(lengths, cu, total, B, H, L, item_rows(kind), ws);
   return cudaGetLastError();
 }
 

@@ -60,6 +60,11 @@ def test_bad_arguments_rejected_before_any_device_work():
     # negative sizes
     assert lib.sigattn_fwd(null, null, null, null, lens, -1, 1, 64, 64, ws, 4096, null) == 1
     assert lib.sigattn_plan(lens, 1, 1, 64, 64, 7, ws, 4096, null) == 1
+    # packed layout: null cu_seqlens, unsupported d, total < 1, too many tokens
+    for fn, nptr in ((lib.sigattn_fwd_varlen, 4), (lib.sigattn_bwd_dq_varlen, 5), (lib.sigattn_bwd_dkdv_varlen, 6)):
+        ptrs = [null] * nptr
+        assert fn(*ptrs, null, 1, 1, 64, 64, 64, null, 0, null) == 1
+        assert fn(*ptrs, lens, 1, 1, 64, 64, 96, ws, 4096, null) == 2
 
 
 @pytest.mark.parametrize("kind", [0, 1, 2])
