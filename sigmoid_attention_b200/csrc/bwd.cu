@@ -476,12 +476,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const int c = g + 2 * i;
           const bool second = c >= D / 32;
           const int col = (second ? c - D / 32 : c) * 32;
-          uint4* dst = reinterpret_cast<uint4*>((second ? out2 : out1) + row_off + col);
           if (valid_row) {
-#pragma unroll
-            for (int w4 = 0; w4 < 4; ++w4)
-              dst[w4] = make_uint4(packed[i][4 * w4], packed[i][4 * w4 + 1], packed[i][4 * w4 + 2],
-                                   packed[i][4 * w4 + 3]);
+            store_row64B((second ? out2 : out1) + row_off + col, packed[i]);
           } else {
             store_zero32((second ? out2 : out1) + row_off + col);
           }

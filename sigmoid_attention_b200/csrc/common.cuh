@@ -149,22 +149,40 @@ __device__ __forceinline__ float sigmoid_from_score(float s, float half_scale, f
   return fmaf(t, 0.5f, 0.5f);
 }
 
-// Convert 32 fp32 accumulator values (times `mul`) to bf16 and store them.
-__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul) {
-  uint4* p = reinterpret_cast<uint4*>(dst);
+// Store 64 bytes (one row's 32 bf16 values, packed in pairs) at dst, which is
+// 16-byte aligned. An epilogue lane owns one row, so a warp's store touches 32
+// rows; 32-byte stores halve the number of such instructions when dst is
+// 32-byte aligned (warp-uniform: row strides are multiples of 32 bytes).
+__device__ __forceinline__ void store_row64B(void* dst, const uint32_t (&w)[16]) {
+  if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    p[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q + 0]) * mul, __uint_as_float(v[8 * q + 1]) * mul),
-                      pack_bf16x2(__uint_as_float(v[8 * q + 2]) * mul, __uint_as_float(v[8 * q + 3]) * mul),
-                      pack_bf16x2(__uint_as_float(v[8 * q + 4]) * mul, __uint_as_float(v[8 * q + 5]) * mul),
-                      pack_bf16x2(__uint_as_float(v[8 * q + 6]) * mul, __uint_as_float(v[8 * q + 7]) * mul));
+    for (int h = 0; h < 2; ++h)
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                       reinterpret_cast<uint8_t*>(dst) + 32 * h),
+                   "r"(w[8 * h]), "r"(w[8 * h + 1]), "r"(w[8 * h + 2]), "r"(w[8 * h + 3]), "r"(w[8 * h + 4]),
+                   "r"(w[8 * h + 5]), "r"(w[8 * h + 6]), "r"(w[8 * h + 7])
+                   : "memory");
+  } else {
+    uint4* p = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) p[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
   }
 }
 
-__device__ __forceinline__ void store_zero32(__nv_bfloat16* dst) {
-  uint4* p = reinterpret_cast<uint4*>(dst);
+// Convert 32 fp32 accumulator values (times `mul`) to bf16 and store them.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul) {
+  uint32_t w[16];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) p[q] = make_uint4(0, 0, 0, 0);
+  for (int e = 0; e < 16; ++e)
+    w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+  store_row64B(dst, w);
+}
+
+__device__ __forceinline__ void store_zero32(__nv_bfloat16* dst) {
+  uint32_t w[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) w[e] = 0u;
+  store_row64B(dst, w);
 }
 
 // Launch `kernel` so that it may start while the previous kernel in `stream` is

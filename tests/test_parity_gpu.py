@@ -176,6 +176,38 @@ def test_full_size_workloads_sampled(name):
     _sampled(workloads.WORKLOADS[name])
 
 
+def test_maximum_batch_of_short_sequences():
+    # SIGATTN_MAX_BATCH sequences in one call (the plan sorts them in one CTA), every element compared.
+    B, H, L, d = 4096, 1, 64, 64
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 61)
+    lengths = workloads.random_lengths(B, L, 61, lo=0)
+    check_full(q, k, v, dout, lengths)
+
+
+def test_long_single_sequence_sampled():
+    # One 65536-token sequence at d = 128: 512 column blocks per item, 4.3e9 valid pairs.
+    B, H, L, d = 1, 1, 65536, 128
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 62)
+    lens = np.array([L], dtype=np.int32)
+    o, dq, dk, dv = run_gpu(q, k, v, dout, lens)
+    for t in (o, dq, dk, dv):
+        assert torch.isfinite(t).all()
+    rng = np.random.default_rng(62)
+    row = np.concatenate([[0, L - 1], rng.integers(0, L, 10)])
+    bh = np.zeros_like(row)
+    for name, got, tol in (("o", o, FWD_REL), ("dq", dq, BWD_REL), ("dk", dk, BWD_REL), ("dv", dv, BWD_REL)):
+        ref = oracle.rows(name, q, k, v, dout, lens, bh, row)
+        g = got.reshape(L, d)[row].numpy()
+        assert rel_l2(g, ref) <= tol, (name, rel_l2(g, ref))
+
+
+def test_single_token_sequences_d128():
+    # n = 1: bias ln 1 = 0, O_0 = sigma(q.k / sqrt(d)) v
+    B, H, L, d = 3, 2, 128, 128
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 63)
+    check_full(q, k, v, dout, [1, 1, 0])
+
+
 def test_autograd_function_matches_direct_calls():
     B, H, L, d = 2, 2, 256, 64
     q, k, v, dout = workloads.make_inputs(B, H, L, d, 31)
