@@ -247,10 +247,17 @@ def run_gpu(args, w):
     flops_fwd = w.fwd_flops()
     flops_bwd = w.bwd_flops()
     pairs = flops_fwd / (4.0 * w.d)
+    packed = args.layout == "packed"
+    if packed:
+        # Valid tokens only, back to back: [total, H, d] and cu_seqlens [B + 1].
+        q, k, v, dout = (torch.cat([t[b, :, :int(n)].permute(1, 0, 2) for b, n in enumerate(lengths.tolist())])
+                         .contiguous() for t in (q, k, v, dout))
+        lengths = torch.cat([torch.zeros(1, dtype=torch.int32), torch.cumsum(lengths, 0).to(torch.int32)])
+        max_seqlen = max(1, int(w.lengths().max()))
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, dout))
     lens = lengths.to(dev)
     o, dq, dk, dv = (torch.empty_like(qd) for _ in range(4))
-    ws = sa.make_workspace(w.B, w.H, w.L, w.d, dev)
+    ws = sa.make_workspace(w.B, w.H, max_seqlen if packed else w.L, w.d, dev)
     stream = torch.cuda.current_stream(dev)
     tensor_bytes = qd.numel() * 2
     footprint = 8 * tensor_bytes
@@ -260,13 +267,22 @@ def run_gpu(args, w):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        sa.sigattn_fwd(qd, kd, vd, o, lens, ws, stream)
+        if packed:
+            sa.sigattn_fwd_varlen(qd, kd, vd, o, lens, max_seqlen, ws, stream)
+        else:
+            sa.sigattn_fwd(qd, kd, vd, o, lens, ws, stream)
         if ev is not None:
             ev[1].record(stream)
-        sa.sigattn_bwd_dq(qd, kd, vd, dod, dq, lens, ws, stream)
+        if packed:
+            sa.sigattn_bwd_dq_varlen(qd, kd, vd, dod, dq, lens, max_seqlen, ws, stream)
+        else:
+            sa.sigattn_bwd_dq(qd, kd, vd, dod, dq, lens, ws, stream)
         if ev is not None:
             ev[2].record(stream)
-        sa.sigattn_bwd_dkdv(qd, kd, vd, dod, dk, dv, lens, ws, stream)
+        if packed:
+            sa.sigattn_bwd_dkdv_varlen(qd, kd, vd, dod, dk, dv, lens, max_seqlen, ws, stream)
+        else:
+            sa.sigattn_bwd_dkdv(qd, kd, vd, dod, dk, dv, lens, ws, stream)
         if ev is not None:
             ev[3].record(stream)
 
@@ -350,8 +366,11 @@ def run_gpu(args, w):
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_s * 1e3 / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {**w.describe(), "valid_pairs_per_head": pairs / w.H,
-                   "step": "sigattn_fwd + sigattn_bwd_dq + sigattn_bwd_dkdv (each: plan + compute kernel)",
+        "config": {**w.describe(), "layout": args.layout, "valid_pairs_per_head": pairs / w.H,
+                   "step": ("sigattn_fwd_varlen + sigattn_bwd_dq_varlen + sigattn_bwd_dkdv_varlen "
+                            "(each: plan + compute kernel)") if packed else
+                           ("sigattn_fwd + sigattn_bwd_dq + sigattn_bwd_dkdv "
+                            "(each: plan + compute kernel + padded-row zero fill)"),
                    "flops": "valid pairs only: 4*d fwd + 10*d bwd per pair",
                    "parallelism": f"replica per GPU x{world} (independent batches)",
                    "l2": ("flushed between steps (footprint %.0f MB)" % (footprint / 1e6)) if flush else
@@ -365,7 +384,7 @@ def run_gpu(args, w):
                      "traffic": _traffic(dominant, w.name)},
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": (6 if packed else 9) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -387,6 +406,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="dense_d128", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--layout", default="padded", choices=["padded", "packed"],
+                    help="padded [B,H,Lmax,d] tensors, or the workload's valid tokens packed as [total,H,d]")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     args = ap.parse_args(argv)
     if args.warmup < 3:
