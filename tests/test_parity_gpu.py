@@ -81,6 +81,33 @@ def test_small_cases_elementwise(B, H, L, d, lengths, seed):
     check_full(q, k, v, dout, lengths)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_wide_score_range(d):
+    # Q and K scaled by 4 (exact in bf16): scores x = s/sqrt(d) - ln n spread over about +-50,
+    # so sigma is exercised deep in both tails as well as in the middle.
+    # Most weights saturate at 0 or 1, so |O| reaches 15-30 and the fixed 2e-2 element bound (meant
+    # for N(0,1) inputs, |O| < ~1) is below the output's own bf16 ulp. The element bound here follows
+    # the arithmetic instead: P is rounded to bf16 before the PV product (relative error <= 2^-9 per
+    # weight, coherent for weights just below 1), so |dO_i| <= 2^-9 sum_j P_ij |V_j| plus the output's
+    # own rounding (2^-9 |O_i|, doubled for the fp32 accumulation) plus a small absolute term.
+    B, H, L = 2, 2, 300
+    lengths = [300, 171]
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 71)
+    q, k = q * 4, k * 4
+    o, dq, dk, dv = run_gpu(q, k, v, dout, lengths)
+    for t in (o, dq, dk, dv):
+        assert torch.isfinite(t).all()
+        check_padded_zero(t, lengths)
+    o_ref = oracle.forward(q, k, v, lengths)
+    dq_ref, dk_ref, dv_ref = oracle.backward(q, k, v, dout, lengths)
+    assert rel_l2(o, o_ref) <= FWD_REL, rel_l2(o, o_ref)
+    weight_abs_v = oracle.forward(q, k, v.abs(), lengths)  # sum_j P_ij |V_j|, exact
+    bound = 2 ** -9 * weight_abs_v + 2 ** -8 * np.abs(o_ref) + 1e-3
+    assert (np.abs(o.numpy() - o_ref) <= bound).all(), float((np.abs(o.numpy() - o_ref) / bound).max())
+    for name, got, ref in (("dq", dq, dq_ref), ("dk", dk, dk_ref), ("dv", dv, dv_ref)):
+        assert rel_l2(got, ref) <= BWD_REL, (name, rel_l2(got, ref))
+
+
 def test_tiny_workload_closed_form_zero_query():
     # Q = 0: every valid weight is 1/(1+n), so O_i = sum_{j<n} V_j / (1+n).
     B, H, L, d = 2, 2, 64, 64
