@@ -34,7 +34,10 @@
  *    zero the workspace once after allocating it (cudaMemset); the library
  *    keeps it consistent afterwards.
  *  - stream: a cudaStream_t (NULL = legacy default stream). Calls only
- *    enqueue work: they neither allocate nor synchronise.
+ *    enqueue work: they neither allocate nor synchronise, so a sequence of
+ *    calls can be captured into a CUDA graph and replayed (make one call on
+ *    the device outside the capture first: it sets up per-device kernel
+ *    attributes).
  *  - Return value: a sigattn_status. Argument errors are reported before
  *    anything is enqueued. A kernel-side timeout (a bounded wait that gave up)
  *    is recorded in the workspace and surfaces through sigattn_read_error.
