@@ -50,12 +50,15 @@ def _peaks():
 
 
 def _csrc_hash() -> str:
+    """Hash of the kernel sources with // comments and blank lines removed, so
+    that the committed ncu traffic stays tied to the code, not to its comments."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sigmoid_attention_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                code = [line.split("//", 1)[0].rstrip() for line in f]
+            h.update(name.encode() + "\n".join(line for line in code if line).encode())
     return h.hexdigest()[:16]
 
 

@@ -34,8 +34,10 @@
 // leave room in the 512 TMEM columns only for 64-column S and dP regions:
 //   XS [0,BN) XdP [BN,2BN) P [2BN,2.5BN) dS [2.5BN,3BN) A1 [3BN,3BN+D) A2 after.
 // Warps: 0-7 epilogue (warps 4g..4g+3 take columns [g BN/2, (g+1) BN/2) of
-// each block), 8 TMA producer, 9 S issuer (owns TMEM), 10 dP issuer, 11 A1
-// issuer, 12 A2 issuer (dK/dV only).
+// each block), 8 TMA producer (also claims the work items and passes them on
+// through the shared-memory item ring), 9 S issuer (owns TMEM), 10 dP issuer,
+// 11 A1 issuer, 12 A2 issuer (dK/dV only). PACKED selects the input layout, as
+// in the forward kernel.
 #include "common.cuh"
 
 namespace sigattn {

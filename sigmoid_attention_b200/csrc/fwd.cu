@@ -11,7 +11,10 @@
 //   warps 0-7   epilogue for query tile 0 (TMEM lanes 0..127 = its 128 rows):
 //               warps 0-3 key columns 0-63, warps 4-7 key columns 64-127
 //   warps 8-15  epilogue for query tile 1, split the same way
-//   warp  16    TMA producer: Q tiles once per item, then a ring of K and V tiles
+//   warp  16    TMA producer: claims work items (first blockIdx.x, then from the
+//               workspace counter) and hands them to the other warps through
+//               the shared-memory item ring; Q tiles once per item, then a ring
+//               of K and V tiles
 //   warps 17,18 one tcgen05.mma issuer per query tile (warp 17 also owns TMEM).
 // A single thread issues a tcgen05.mma only every ~100 cycles, which is more
 // than a 128x128x16 product takes, so each tile has its own issuing thread;
@@ -29,6 +32,9 @@
 // done): each has the MUFU pipe to itself while the tensor core works on the
 // other tile, instead of both tiles running in phase.
 // TMEM: S/P of tile t at columns [128t, 128t+128), O of tile t at 256 + t*D.
+// PACKED selects the input layout (padded [B][H][Lmax][d] or packed
+// [total][H][d]); it changes only the TMA coordinates and output row addresses
+// (RowMap), so both layouts run the same arithmetic in the same order.
 #include "common.cuh"
 
 namespace sigattn {
