@@ -160,6 +160,22 @@ def test_device_plan_bit_exact(kind):
     assert got == expect
 
 
+@pytest.mark.parametrize("kind", [0, 1, 2])
+def test_device_plan_bit_exact_at_maximum_batch(kind):
+    # 4096 sequences (the plan's rank sort and 32-wide scan over many rounds), many ties, some empty.
+    H, L, d = 2, 700, 64
+    lens_np = workloads.random_lengths(4096, L, 90 + kind, lo=0)
+    lens = torch.from_numpy(lens_np).cuda()
+    ws = sa.make_workspace(len(lens_np), H, L, d)
+    sa.sigattn_plan(lens, len(lens_np), H, L, d, kind, ws)
+    torch.cuda.synchronize()
+    dev_items = sa.read_plan(ws)
+    assert torch.equal(dev_items, sa.sigattn_plan_host(lens_np, H, L, kind))
+    got = sorted((int(bh) // H, int(bh) % H, int(m)) for bh, m in dev_items.tolist())
+    expect = [tuple(t) for t in oracle.tiles(lens_np, H, L, sa.sigattn_block_rows(kind)).tolist()]
+    assert got == expect
+
+
 def test_invalid_length_flags_error_and_zeros_sequence():
     B, H, L, d = 2, 1, 64, 64
     q, k, v, dout = workloads.make_inputs(B, H, L, d, 23)
