@@ -55,7 +55,13 @@ struct FwdCfg {
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;     // slack for 1024-byte alignment
   static constexpr int TM_S = 0;
   static constexpr int TM_O = 256;
+  // At D = 64 the 512 TMEM columns leave room for P in its own region (64
+  // columns of bf16 pairs per tile) instead of over S, so S(j+1) need not wait
+  // for PV(j), and all 16 epilogue warps take each tile's sigmoid pass: SEP_P.
+  static constexpr bool SEP_P = (D == 64);
+  static constexpr int TM_P = TM_O + 2 * D;
   static constexpr int TMEM_COLS = 512;
+  static_assert(!SEP_P || TM_P + 128 <= TMEM_COLS, "TMEM budget");
   static constexpr int EPI_WARPS = 16;
   static constexpr int THREADS = (EPI_WARPS + 3) * 32;
 };
@@ -67,6 +73,8 @@ struct FwdBarriers {
   uint64_t v_full[VST], v_empty[VST];
   uint64_t s_full[2], p_full[4], o_full[2], o_empty[2];
   uint64_t epi_done[2];  // tile t's warps finished their sigmoid pass over a block
+  uint64_t s_read[2];    // SEP_P: the epilogue copied tile t's S out of TMEM (S region free)
+  uint64_t pv_done[2];   // SEP_P: tile t's PV products of a block completed (P region free)
   uint64_t drain[2];
   ItemRing ring;
   uint32_t tmem_base;
@@ -99,8 +107,12 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     for (int s = 0; s < C::VST; ++s) { mbar_init(&bar.v_full[s], 1); mbar_init(&bar.v_empty[s], 2); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar.s_full[t], 1);
-      mbar_init(&bar.p_full[2 * t], 4);
-      mbar_init(&bar.p_full[2 * t + 1], 4);
+      // P of a key half: 4 warps (one per lane quadrant), or with SEP_P the 8
+      // warps that cover its two 32-column chunks.
+      mbar_init(&bar.p_full[2 * t], C::SEP_P ? 8 : 4);
+      mbar_init(&bar.p_full[2 * t + 1], C::SEP_P ? 8 : 4);
+      mbar_init(&bar.s_read[t], C::EPI_WARPS);
+      mbar_init(&bar.pv_done[t], 1);
       mbar_init(&bar.o_full[t], 1);
       mbar_init(&bar.o_empty[t], 8);
     }
@@ -205,6 +217,12 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       constexpr uint64_t kTile = C::TILE_BYTES >> 4;
       const uint32_t tm_s = tmem + C::TM_S + t * 128;
       const uint32_t tm_o = tmem + C::TM_O + t * D;
+      // P of key half h: over the first 32 columns of S's half, or (SEP_P) in
+      // its own region, 32 columns per half.
+      const uint32_t tm_p = C::SEP_P ? tmem + C::TM_P + t * 64 : tm_s;
+      constexpr int kPHalf = C::SEP_P ? 32 : 64;
+      uint32_t srph = 0;
+      bool s_pending = false;  // SEP_P: an S was issued whose copy-out has not been awaited
 
       auto issue_s = [&](uint32_t ks) {
         const uint64_t b0 = d_k + ks * kTile;
@@ -220,10 +238,19 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
         const uint64_t b0 = d_v + vs * kTile + ((h * 64 * 128) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tm_o, tm_s + h * 64 + kk * 8, b0 + ((kk * 2048) >> 4), idesc_o, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tm_o, tm_p + h * kPHalf + kk * 8, b0 + ((kk * 2048) >> 4), idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
       auto advance_k = [&]() { if (++kst == C::KST) { kst = 0; kph ^= 1; } };
       auto advance_v = [&]() { if (++vst == C::VST) { vst = 0; vph ^= 1; } };
+      // SEP_P: before an S product overwrites the S region, the epilogue must
+      // have copied out the previous S of this tile.
+      auto wait_s_free = [&]() -> bool {
+        if (!C::SEP_P || !s_pending) return true;
+        if (!mbar_wait(&bar.s_read[t], srph, abort_flag, ws, 118)) return false;
+        srph ^= 1;
+        s_pending = false;
+        return true;
+      };
 
       uint32_t ist = 0, iph = 0;
       while (ok) {
@@ -255,8 +282,10 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
         if (!(ok = mbar_wait(&bar.q_full, qph, abort_flag, ws, 111))) break;
         qph ^= 1;
         if (!(ok = mbar_wait(&bar.k_full[kst], kph, abort_flag, ws, 112))) break;
+        if (!(ok = wait_s_free())) break;
         tc_fence_after();
         issue_s(kst);
+        s_pending = true;
         mma_commit(&bar.s_full[t]);
         if (nkb == 1) mma_commit(&bar.q_empty);
         mma_commit(&bar.k_empty[kst]);
@@ -264,6 +293,22 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
 
         for (int j = 0; ok && j < nkb; ++j) {
           const bool has_next = (j + 1 < nkb);
+          // S(j+1) goes first when P has its own region (as soon as the
+          // epilogue has copied S(j) out); otherwise it overwrites P(j) and
+          // must follow PV(j).
+          auto next_s = [&]() -> bool {
+            if (!mbar_wait(&bar.k_full[kst], kph, abort_flag, ws, 116)) return false;
+            if (!wait_s_free()) return false;
+            tc_fence_after();
+            issue_s(kst);
+            s_pending = true;
+            mma_commit(&bar.s_full[t]);
+            if (j + 2 == nkb) mma_commit(&bar.q_empty);
+            mma_commit(&bar.k_empty[kst]);
+            advance_k();
+            return true;
+          };
+          if (C::SEP_P && has_next && !(ok = next_s())) break;
           if (!(ok = mbar_wait(&bar.v_full[vst], vph, abort_flag, ws, 113))) break;
           for (int h = 0; h < 2; ++h) {
             if (!(ok = mbar_wait(&bar.p_full[2 * t + h], pph[h], abort_flag, ws, 114))) break;
@@ -278,15 +323,8 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           if (!ok) break;
           mma_commit(&bar.v_empty[vst]);
           advance_v();
-          if (has_next) {
-            if (!(ok = mbar_wait(&bar.k_full[kst], kph, abort_flag, ws, 116))) break;
-            tc_fence_after();
-            issue_s(kst);
-            mma_commit(&bar.s_full[t]);
-            if (j + 2 == nkb) mma_commit(&bar.q_empty);
-            mma_commit(&bar.k_empty[kst]);
-            advance_k();
-          }
+          if (C::SEP_P) mma_commit(&bar.pv_done[t]);
+          if (!C::SEP_P && has_next && !(ok = next_s())) break;
         }
         if (!ok) break;
         mma_commit(&bar.o_full[t]);
@@ -295,6 +333,91 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       int never = 0;
       mma_commit(&bar.drain[t]);
       mbar_wait(&bar.drain[t], 0, &never, ws, 119);
+    }
+  } else if constexpr (C::SEP_P) {
+    // ------------------------------------------------- epilogue (D = 64, SEP_P)
+    // All 16 warps take each tile's sigmoid pass in turn (tile 0, then tile 1,
+    // block by block), so the two tiles' passes never compete for MUFU and
+    // each has four warps per scheduler to hide the TMEM latencies. Warp w
+    // reads TMEM lane quadrant w & 3 and key columns [32c, 32c + 32), c = w >> 2;
+    // its P (bf16 pairs) goes to columns [16c, 16c + 16) of the tile's P region.
+    // At the end of an item warp w reads out tile c >> 1, output columns
+    // [32 (c & 1), 32 (c & 1) + 32).
+    const int c = warp >> 2;
+    const int r = ((warp & 3) << 5) + lane;        // row within a tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
+    const int ot = c >> 1, oc = c & 1;
+    constexpr float half_scale = 0.5f * Scale<D>::value;
+    uint32_t sph[2] = {0, 0}, oph[2] = {0, 0}, pvph[2] = {0, 0};
+    bool pv_pending[2] = {false, false};  // a P of the tile was written whose PV has not been awaited
+    bool ok = true;
+    uint32_t ist = 0, iph = 0;
+    while (ok) {
+      Item item;
+      if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 120))) break;
+      __syncwarp();
+      ring_release(bar.ring, ist, iph, lane == 0);
+      if (item.n < 0) break;
+      const int n = item.n;
+      const int row_base = item.blk * (C::BM * C::NQ);
+      const int ntiles = (row_base + C::BM < n) ? 2 : 1;
+      const int nkb = ceil_div(n, C::BN);
+      const float half_bias = -0.5f * __logf(static_cast<float>(n));
+      for (int j = 0; ok && j < nkb; ++j) {
+        const int valid = n - (j * C::BN + 32 * c);  // columns < valid are real keys
+        for (int t = 0; t < ntiles; ++t) {
+          if (!(ok = mbar_wait(&bar.s_full[t], sph[t], abort_flag, ws, 121))) break;
+          sph[t] ^= 1;
+          tc_fence_after();
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + C::TM_S + t * 128 + 32 * c, a);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.s_read[t]);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float p0 = sigmoid_from_score(__uint_as_float(a[2 * e]), half_scale, half_bias);
+            float p1 = sigmoid_from_score(__uint_as_float(a[2 * e + 1]), half_scale, half_bias);
+            if (valid < 32) {
+              p0 = (2 * e < valid) ? p0 : 0.f;
+              p1 = (2 * e + 1 < valid) ? p1 : 0.f;
+            }
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          // The P region is free once the tile's previous PV products completed.
+          if (pv_pending[t]) {
+            if (!(ok = mbar_wait(&bar.pv_done[t], pvph[t], abort_flag, ws, 124))) break;
+            pvph[t] ^= 1;
+          }
+          pv_pending[t] = true;
+          tc_fence_after();
+          tmem_st16(tmem + lane_off + C::TM_P + t * 64 + 16 * c, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.p_full[2 * t + (c >> 1)]);
+        }
+      }
+      if (!ok) break;
+      const int row = row_base + ot * C::BM + r;
+      __nv_bfloat16* orow = out + rm.offset(item, PACKED ? item.bh % H : 0, row, D) + 32 * oc;
+      if (ot >= ntiles) {  // tile fully padded: its rows of O are zero (padded layout)
+        if (rm.writes(row, n)) store_zero32(orow);
+        continue;
+      }
+      if (!(ok = mbar_wait(&bar.o_full[ot], oph[ot], abort_flag, ws, 122))) break;
+      oph[ot] ^= 1;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + C::TM_O + ot * D + 32 * oc, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.o_empty[ot]);
+      if (rm.writes(row, n)) {
+        if (row < n) store_row32(orow, v, 1.0f);
+        else store_zero32(orow);
+      }
     }
   } else {
     // ------------------------------------------------------------- epilogue
