@@ -24,6 +24,7 @@ __all__ = [
     "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
     "sigattn_fwd_varlen", "sigattn_bwd_dq_varlen", "sigattn_bwd_dkdv_varlen",
     "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
+    "SigmoidAttentionVarlenFunction", "sigmoid_attention_varlen",
 ]
 
 KIND_FWD, KIND_DQ, KIND_DKDV = 0, 1, 2
@@ -297,3 +298,32 @@ class SigmoidAttentionFunction(torch.autograd.Function):
 
 def sigmoid_attention(q, k, v, lengths) -> torch.Tensor:
     return SigmoidAttentionFunction.apply(q, k, v, lengths)
+
+
+class SigmoidAttentionVarlenFunction(torch.autograd.Function):
+    """Autograd wrapper of the packed-layout calls: q, k, v are [total, H, d]
+    with sequences back to back as given by cu_seqlens (int32 [B + 1])."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, cu_seqlens, max_seqlen):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        _, H, d = _packed_dims(q)
+        ws = make_workspace(cu_seqlens.numel() - 1, H, max_seqlen, d, q.device)
+        o = torch.empty_like(q)
+        sigattn_fwd_varlen(q, k, v, o, cu_seqlens, max_seqlen, ws)
+        ctx.save_for_backward(q, k, v, cu_seqlens, ws)
+        ctx.max_seqlen = max_seqlen
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, cu_seqlens, ws = ctx.saved_tensors
+        do = do.contiguous()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        sigattn_bwd_dq_varlen(q, k, v, do, dq, cu_seqlens, ctx.max_seqlen, ws)
+        sigattn_bwd_dkdv_varlen(q, k, v, do, dk, dv, cu_seqlens, ctx.max_seqlen, ws)
+        return dq, dk, dv, None, None
+
+
+def sigmoid_attention_varlen(q, k, v, cu_seqlens, max_seqlen: int) -> torch.Tensor:
+    return SigmoidAttentionVarlenFunction.apply(q, k, v, cu_seqlens, int(max_seqlen))

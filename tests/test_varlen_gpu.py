@@ -160,3 +160,17 @@ def test_full_size_workload_packed_equals_padded(name):
     packed, _, _ = run_packed(q, k, v, dout, lengths)
     for nm, a, b in zip(("o", "dq", "dk", "dv"), padded, packed):
         assert torch.equal(a, b), (name, nm)
+
+
+def test_varlen_autograd_matches_direct_calls():
+    B, H, L, d = 3, 2, 300, 64
+    lengths = [300, 90, 129]
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 48)
+    (_, raw, cu) = run_packed(q, k, v, dout, lengths)
+    dev = torch.device("cuda")
+    qp, kp, vp, dop = (pack(t, lengths)[0].to(dev) for t in (q, k, v, dout))
+    qp, kp, vp = (t.requires_grad_(True) for t in (qp, kp, vp))
+    o = sa.sigmoid_attention_varlen(qp, kp, vp, cu.to(dev), max(lengths))
+    o.backward(dop)
+    for got, ref in zip((o.detach(), qp.grad, kp.grad, vp.grad), raw):
+        assert torch.equal(got.cpu(), ref)
