@@ -1,6 +1,8 @@
 // api.cu -- the C ABI (include/sigattn.h): argument checks, TMA tensor maps and
-// the launches of the plan and compute kernels. No allocation, no host sync
-// (except in sigattn_read_error, which exists to synchronise).
+// the launches of each call's kernels (plan; compute, with a programmatic
+// dependency on the plan; for the padded layout the zero fill of uncovered
+// output rows). No allocation, no host sync (except in sigattn_read_error,
+// which exists to synchronise).
 #include <climits>
 #include <cstdio>
 #include <cstring>
