@@ -41,6 +41,8 @@
  *  - Return value: a sigattn_status. Argument errors are reported before
  *    anything is enqueued. A kernel-side timeout (a bounded wait that gave up)
  *    is recorded in the workspace and surfaces through sigattn_read_error.
+ *  - Outputs must not overlap the inputs or each other: the kernels read
+ *    input tiles while other tiles of the outputs are being written.
  *  - Ownership: the library keeps no pointer after a call returns.
  */
 #ifndef SIGATTN_H_
