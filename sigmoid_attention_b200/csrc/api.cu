@@ -22,7 +22,7 @@ cudaError_t launch_fwd(int d, bool packed, const CUtensorMap& tq, const CUtensor
                        void* o, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_dq(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                           const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L, int num_sms,
-                          cudaStream_t stream);
+                          const int* fill_lengths, cudaStream_t stream);
 cudaError_t launch_bwd_dkdv(int d, bool packed, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                             const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int L, int num_sms,
                             cudaStream_t stream);
@@ -224,10 +224,9 @@ int sigattn_bwd_dq(const void* q, const void* k, const void* v, const void* dout
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
   st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_DQ, ws, s));
-  if (st == SIGATTN_OK)
-    st = cuda_status(launch_bwd_dq(d, false, tq, tdo, tk, tv, dq, ws, B, H, Lmax, info.num_sms, s));
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_DQ, dq, nullptr, info.num_sms, s));
+  // The dQ kernel zeroes dQ's uncovered padded rows itself.
+  return cuda_status(launch_bwd_dq(d, false, tq, tdo, tk, tv, dq, ws, B, H, Lmax, info.num_sms, lengths, s));
 }
 
 int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
@@ -290,7 +289,7 @@ int sigattn_bwd_dq_varlen(const void* q, const void* k, const void* v, const voi
   int* ws = static_cast<int*>(workspace);
   st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_DQ, ws, s));
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_bwd_dq(d, true, tq, tdo, tk, tv, dq, ws, B, H, max_seqlen, info.num_sms, s));
+  return cuda_status(launch_bwd_dq(d, true, tq, tdo, tk, tv, dq, ws, B, H, max_seqlen, info.num_sms, nullptr, s));
 }
 
 int sigattn_bwd_dkdv_varlen(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,

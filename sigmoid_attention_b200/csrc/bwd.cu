@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_r1, const __grid_constant__ CUtensorMap tm_r2,
                const __grid_constant__ CUtensorMap tm_c1, const __grid_constant__ CUtensorMap tm_c2,
                __nv_bfloat16* __restrict__ out1, __nv_bfloat16* __restrict__ out2,
-               int* __restrict__ ws, int H, int L) {
+               int* __restrict__ ws, int H, int L, const int* __restrict__ fill_lengths, int B, int fill_parts) {
   using C = BwdCfg<D, KV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ BwdBarriers<C::ST1, C::ST2> bar;
@@ -488,6 +488,21 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     }
   }
 
+  // dQ over padded inputs: the rows no item covers are zeroed here, in the
+  // kernel's tail. Each warp joins once its role is done and claims fill units
+  // from the workspace counter, so the CTAs that run out of items first do
+  // most of it.
+  if (fill_lengths != nullptr) {
+    const long long units = static_cast<long long>(B) * H * fill_parts;
+    while (true) {
+      int u = 0;
+      if (lane == 0) u = atomicAdd(ws + kHdrFill, 1);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (u >= units) break;
+      zero_fill_unit(fill_lengths, H, L, D, C::BM, fill_parts, u, lane, out1, nullptr);
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == kSWarp) {
@@ -499,7 +514,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
 template <int D, bool KV, bool PACKED>
 cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
                             const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
-                            cudaStream_t stream) {
+                            const int* fill_lengths, cudaStream_t stream) {
   using C = BwdCfg<D, KV>;
   static bool configured[64] = {};
   int dev = 0;
@@ -512,32 +527,38 @@ cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const 
   }
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kBwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
+  const int parts = zero_fill_parts(static_cast<long long>(B) * H, num_sms);
   return launch_programmatic(bwd_kernel<D, KV, PACKED>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2,
-                             c1, c2, static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), ws, H, L);
+                             c1, c2, static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), ws, H, L,
+                             fill_lengths, B, parts);
 }
 
 template <bool KV>
 cudaError_t launch_bwd(int d, bool packed, const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
                        const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
-                       cudaStream_t stream) {
+                       const int* fill_lengths, cudaStream_t stream) {
   if (packed) {
-    if (d == 64) return launch_bwd_impl<64, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, stream);
-    return launch_bwd_impl<128, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, stream);
+    if (d == 64)
+      return launch_bwd_impl<64, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
+    return launch_bwd_impl<128, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
   }
-  if (d == 64) return launch_bwd_impl<64, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, stream);
-  return launch_bwd_impl<128, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, stream);
+  if (d == 64)
+    return launch_bwd_impl<64, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
+  return launch_bwd_impl<128, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
 }
 
+// fill_lengths: the padded layout's lengths, so that the dQ kernel zeroes the
+// uncovered rows of dQ itself (nullptr for the packed layout).
 cudaError_t launch_bwd_dq(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                           const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L, int num_sms,
-                          cudaStream_t stream) {
-  return launch_bwd<false>(d, packed, tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, num_sms, stream);
+                          const int* fill_lengths, cudaStream_t stream) {
+  return launch_bwd<false>(d, packed, tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, num_sms, fill_lengths, stream);
 }
 
 cudaError_t launch_bwd_dkdv(int d, bool packed, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                             const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int L, int num_sms,
                             cudaStream_t stream) {
-  return launch_bwd<true>(d, packed, tk, tv, tq, tdo, dk, dv, ws, B, H, L, num_sms, stream);
+  return launch_bwd<true>(d, packed, tk, tv, tq, tdo, dk, dv, ws, B, H, L, num_sms, nullptr, stream);
 }
 
 }  // namespace sigattn

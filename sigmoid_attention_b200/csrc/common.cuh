@@ -2,6 +2,7 @@
 // and backward kernels of the sigmoid-attention library.
 #pragma once
 
+#include <algorithm>
 #include <cstdint>
 #include <utility>
 #include <cuda_bf16.h>
@@ -147,6 +148,31 @@ struct Scale<128> {
 __device__ __forceinline__ float sigmoid_from_score(float s, float half_scale, float half_bias) {
   const float t = tanh_approx(fmaf(s, half_scale, half_bias));
   return fmaf(t, 0.5f, 0.5f);
+}
+
+// Zero one unit of the output rows that no work item covers: rows
+// [ceil(n_b/rows)*rows, L) of slice u / parts are cut into `parts` interleaved
+// shares of 16-byte chunks, and this warp writes share u % parts of out0 (and
+// out1).
+__device__ __forceinline__ void zero_fill_unit(const int* lengths, int H, int L, int d, int rows, int parts,
+                                               long long u, int lane, __nv_bfloat16* out0, __nv_bfloat16* out1) {
+  const int slice = static_cast<int>(u / parts);
+  const int part = static_cast<int>(u % parts);
+  const int n = load_len(lengths, slice / H, L);
+  const int cover = min(L, ceil_div(n, rows) * rows);
+  const long long nchunks = static_cast<long long>(L - cover) * (d / 8);  // 16-byte chunks
+  const size_t base = (static_cast<size_t>(slice) * L + cover) * d;
+  uint4* p0 = reinterpret_cast<uint4*>(out0 + base);
+  uint4* p1 = out1 ? reinterpret_cast<uint4*>(out1 + base) : nullptr;
+  for (long long c = static_cast<long long>(part) * 32 + lane; c < nchunks; c += static_cast<long long>(parts) * 32) {
+    p0[c] = make_uint4(0, 0, 0, 0);
+    if (p1) p1[c] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Shares per slice for the zero fill: enough units to spread over the SMs.
+inline int zero_fill_parts(long long slices, int num_sms) {
+  return static_cast<int>(std::max<long long>(1, std::min<long long>(64, (4LL * num_sms + slices - 1) / slices)));
 }
 
 // Store 64 bytes (one row's 32 bf16 values, packed in pairs) at dst, which is

@@ -12,11 +12,12 @@
 //     compute grid takes items round-robin, which spreads the long items over
 //     all SMs first (longest-processing-time-first order);
 //   * rows of the outputs that no item covers (rows >= ceil(n_b/rows)*rows)
-//     are written as exact zeros by fill_kernel, a one-warp-per-CTA kernel
-//     launched right after the compute kernel; for the forward and dK/dV
-//     kernels with a programmatic edge, so that it runs on the registers and
-//     warps the persistent compute CTA leaves free and its HBM writes overlap
-//     the compute-bound kernel instead of preceding it.
+//     are written as exact zeros: after the forward and dK/dV kernels by
+//     fill_kernel, a one-warp-per-CTA kernel launched with a programmatic edge,
+//     so that it runs on the registers and warps the persistent compute CTA
+//     leaves free and its HBM writes overlap the compute-bound kernel; the dQ
+//     kernel zeroes its own in its tail (each warp, once its role is done,
+//     claims fill units from a counter in the workspace header).
 #include <algorithm>
 #include <numeric>
 #include <vector>
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
   if (tid == 0) {
     ws[kHdrCount] = total;
     ws[kHdrNext] = 0;  // the compute kernel's claim counter
+    ws[kHdrFill] = 0;  // the dQ kernel's zero-fill claim counter
   }
   int4* items = reinterpret_cast<int4*>(ws + kHeaderWords);
   for (int i = tid; i < total; i += blockDim.x) {
@@ -136,45 +138,20 @@ cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int
 // the call) completes only after the compute kernel before it.
 __global__ void __launch_bounds__(32) fill_kernel(const int* __restrict__ lengths, int B, int H, int L, int d,
                                                   int rows, int parts, __nv_bfloat16* out0, __nv_bfloat16* out1) {
-  const int lane = threadIdx.x;
-  const int chunks_per_row = d / 8;  // 16-byte chunks
   const long long units = static_cast<long long>(B) * H * parts;
-  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-    const int slice = static_cast<int>(u / parts);
-    const int part = static_cast<int>(u % parts);
-    const int n = load_len(lengths, slice / H, L);
-    const int cover = min(L, ceil_div(n, rows) * rows);
-    const long long nchunks = static_cast<long long>(L - cover) * chunks_per_row;
-    const size_t base = (static_cast<size_t>(slice) * L + cover) * d;
-    uint4* p0 = reinterpret_cast<uint4*>(out0 + base);
-    uint4* p1 = out1 ? reinterpret_cast<uint4*>(out1 + base) : nullptr;
-    for (long long c = static_cast<long long>(part) * 32 + lane; c < nchunks; c += static_cast<long long>(parts) * 32) {
-      p0[c] = make_uint4(0, 0, 0, 0);
-      if (p1) p1[c] = make_uint4(0, 0, 0, 0);
-    }
-  }
+  for (long long u = blockIdx.x; u < units; u += gridDim.x)
+    zero_fill_unit(lengths, H, L, d, rows, parts, u, threadIdx.x, out0, out1);
   grid_dep_wait();
 }
 
-// The fill overlaps the forward and dK/dV kernels. Beside the dQ kernel, whose
-// CTA leaves exactly one warp's worth of registers free, the co-resident fill
-// warps were measured to stream at ~2 GB/s each and to stretch the call 2.5x
-// (B=16, H=12, L=4096, d=64, 75% padding: 0.45 ms against 0.18 ms), so after
-// dQ the fill is an ordinary launch that runs once the compute kernel is done.
+// The fill overlaps the forward and dK/dV kernels (for dQ the compute kernel
+// zeroes its own uncovered rows in its tail, see bwd.cu).
 cudaError_t launch_fill(const int* lengths, int B, int H, int L, int d, int kind, void* out0, void* out1,
                         int num_sms, cudaStream_t stream) {
-  const long long slices = static_cast<long long>(B) * H;
-  const int parts =
-      static_cast<int>(std::max<long long>(1, std::min<long long>(64, (4LL * num_sms + slices - 1) / slices)));
+  const int parts = zero_fill_parts(static_cast<long long>(B) * H, num_sms);
   const int grid = std::max(1, num_sms);
-  const int rows = item_rows(kind);
-  __nv_bfloat16* o0 = static_cast<__nv_bfloat16*>(out0);
-  __nv_bfloat16* o1 = static_cast<__nv_bfloat16*>(out1);
-  if (kind == kKindDq) {
-    fill_kernel<<<grid, 32, 0, stream>>>(lengths, B, H, L, d, rows, parts, o0, o1);
-    return cudaGetLastError();
-  }
-  return launch_programmatic(fill_kernel, dim3(grid), dim3(32), 0, stream, lengths, B, H, L, d, rows, parts, o0, o1);
+  return launch_programmatic(fill_kernel, dim3(grid), dim3(32), 0, stream, lengths, B, H, L, d, item_rows(kind),
+                             parts, static_cast<__nv_bfloat16*>(out0), static_cast<__nv_bfloat16*>(out1));
 }
 
 // Diagnostic: one warp waits, with a bounded wait, on an mbarrier that nothing

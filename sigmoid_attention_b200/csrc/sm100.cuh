@@ -24,6 +24,7 @@ enum : int {
   kHdrErrorSite = 1,  // which wait timed out / which check failed
   kHdrCount = 2,      // number of work items in the list
   kHdrNext = 3,       // work-item claim counter of the compute kernels (zeroed by the plan)
+  kHdrFill = 4,       // zero-fill unit claim counter of the dQ kernel (zeroed by the plan)
   kHeaderWords = 64,  // 256 bytes
 };
 
