@@ -26,7 +26,12 @@
  *  - The scale is 1/sqrt(d) and the bias -ln(n_b) is computed in-kernel; the
  *    bias has no gradient. There is no causal mask.
  *  - Arithmetic: bf16 operands, fp32 accumulation, P (and dS) rounded to bf16
- *    before the second matrix product, outputs rounded to nearest bf16.
+ *    before the second matrix product, outputs rounded to nearest bf16. sigma
+ *    is computed as 1/2 + tanh(x/2)/2 with the hardware tanh (one MUFU
+ *    operation per score) when Lmax <= 65536; above that the bias -ln(n) puts
+ *    most weights below 1e-5, where that route's absolute error becomes a
+ *    relative error of percent size, so calls with a larger Lmax (max_seqlen
+ *    for the packed calls) use 1/(1 + 2^(-x log2 e)) (two MUFU operations).
  *  - workspace: caller-owned device memory of at least
  *    sigattn_workspace_size(B, H, Lmax, d) bytes, 16-byte aligned. Each call
  *    writes its work list there; calls that may run concurrently (different

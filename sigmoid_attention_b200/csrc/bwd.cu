@@ -94,7 +94,8 @@ struct BwdBarriers {
   int abort;
 };
 
-template <int D, bool KV, bool PACKED>
+// ACC: the accurate sigmoid route (calls whose Lmax exceeds kAccurateSigmoidLen).
+template <int D, bool KV, bool PACKED, bool ACC>
 __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_r1, const __grid_constant__ CUtensorMap tm_r2,
                const __grid_constant__ CUtensorMap tm_c1, const __grid_constant__ CUtensorMap tm_c2,
@@ -342,6 +343,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     const uint32_t tXDP1 = tmem + lane_off + C::TM_XDP1 + g * CPW * 32;
     constexpr float scale = Scale<D>::value;
     constexpr float half_scale = 0.5f * scale;
+    constexpr float neg_scale_l2e = -scale * 1.4426950408889634f;
     uint32_t s_ph = 0, free_ph = 0, aph = 0, xb = 0;
     uint32_t dp_ph[2] = {0, 0};
     bool ok = true;
@@ -355,6 +357,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       const int n = item.n;
       const int nb = ceil_div(n, C::BN);
       const float half_bias = -0.5f * __logf(static_cast<float>(n));
+      const float neg_bias_l2e = __log2f(static_cast<float>(n));  // -bias * log2(e)
       for (int j = 0; j < nb; ++j) {
         // ---- S -> P (fp32 kept in registers for dS), bf16 P for dV
         float p[CPW][32];
@@ -371,13 +374,18 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.xs_read);
           const int valid = n - (j * C::BN + g * CPW * 32);  // columns < valid are real tokens
+          auto chunks_p = [&](auto accurate) {
+            constexpr bool kAcc = decltype(accurate)::value;
 #pragma unroll
-          for (int c = 0; c < CPW; ++c)
+            for (int c = 0; c < CPW; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float pe = sigmoid_from_score(__uint_as_float(sv[c][e]), half_scale, half_bias);
-              p[c][e] = (valid >= CPW * 32 || 32 * c + e < valid) ? pe : 0.f;
-            }
+              for (int e = 0; e < 32; ++e) {
+                const float pe =
+                    sigmoid_of<kAcc>(__uint_as_float(sv[c][e]), half_scale, half_bias, neg_scale_l2e, neg_bias_l2e);
+                p[c][e] = (valid >= CPW * 32 || 32 * c + e < valid) ? pe : 0.f;
+              }
+          };
+          chunks_p(std::integral_constant<bool, ACC>{});
         }
         if (KV) {
           if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
@@ -511,7 +519,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   }
 }
 
-template <int D, bool KV, bool PACKED>
+template <int D, bool KV, bool PACKED, bool ACC>
 cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
                             const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
                             const int* fill_lengths, cudaStream_t stream) {
@@ -521,16 +529,28 @@ cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const 
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+        cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED, ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kBwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
   const int parts = zero_fill_parts(static_cast<long long>(B) * H, num_sms);
-  return launch_programmatic(bwd_kernel<D, KV, PACKED>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2,
+  return launch_programmatic(bwd_kernel<D, KV, PACKED, ACC>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2,
                              c1, c2, static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), ws, H, L,
                              fill_lengths, B, parts);
+}
+
+template <int D, bool KV, bool PACKED>
+cudaError_t launch_bwd_acc(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1, const CUtensorMap& c2,
+                           void* out1, void* out2, int* ws, int B, int H, int L, int num_sms, const int* fill_lengths,
+                           cudaStream_t stream) {
+  // No sequence is longer than L, so L decides the sigmoid route for the call.
+  if (L > kAccurateSigmoidLen)
+    return launch_bwd_impl<D, KV, PACKED, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths,
+                                                stream);
+  return launch_bwd_impl<D, KV, PACKED, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths,
+                                               stream);
 }
 
 template <bool KV>
@@ -539,12 +559,12 @@ cudaError_t launch_bwd(int d, bool packed, const CUtensorMap& r1, const CUtensor
                        const int* fill_lengths, cudaStream_t stream) {
   if (packed) {
     if (d == 64)
-      return launch_bwd_impl<64, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
-    return launch_bwd_impl<128, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
+      return launch_bwd_acc<64, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
+    return launch_bwd_acc<128, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
   }
   if (d == 64)
-    return launch_bwd_impl<64, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
-  return launch_bwd_impl<128, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
+    return launch_bwd_acc<64, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
+  return launch_bwd_acc<128, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
 }
 
 // fill_lengths: the padded layout's lengths, so that the dQ kernel zeroes the

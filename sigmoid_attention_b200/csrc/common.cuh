@@ -4,6 +4,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <type_traits>
 #include <utility>
 #include <cuda_bf16.h>
 
@@ -193,6 +194,27 @@ __device__ __forceinline__ void store_row64B(void* dst, const uint32_t (&w)[16])
 #pragma unroll
     for (int q = 0; q < 4; ++q) p[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
   }
+}
+
+// sigma for long sequences. The bias -ln(n) puts the typical weight near 1/n;
+// for n beyond kAccurateSigmoidLen the tanh route computes those weights just
+// above tanh = -1, where the hardware tanh's absolute error becomes a relative
+// error of several percent (measured: O rel-L2 1.1e-2 at n = 2^20). There
+// sigma = 1 / (1 + 2^(-x log2 e)) is used instead: two MUFU operations (ex2,
+// rcp) per score, relative error ~1e-6 everywhere. neg_scale_l2e = -scale *
+// log2(e), neg_bias_l2e = ln(n) * log2(e) = log2(n).
+constexpr int kAccurateSigmoidLen = 65536;
+
+__device__ __forceinline__ float sigmoid_accurate(float s, float neg_scale_l2e, float neg_bias_l2e) {
+  return rcp_approx(1.0f + ex2_approx(fmaf(s, neg_scale_l2e, neg_bias_l2e)));
+}
+
+// ACCURATE (a kernel template parameter, chosen per call from Lmax) selects
+// sigmoid_accurate.
+template <bool ACCURATE>
+__device__ __forceinline__ float sigmoid_of(float s, float half_scale, float half_bias, float neg_scale_l2e,
+                                            float neg_bias_l2e) {
+  return ACCURATE ? sigmoid_accurate(s, neg_scale_l2e, neg_bias_l2e) : sigmoid_from_score(s, half_scale, half_bias);
 }
 
 // Convert 32 fp32 accumulator values (times `mul`) to bf16 and store them.

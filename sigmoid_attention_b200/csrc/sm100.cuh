@@ -275,6 +275,18 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Pack two floats into a bf16x2 word (round to nearest even); `lo` lands in the
 // low 16 bits, which tcgen05 reads as the element with the smaller K index.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

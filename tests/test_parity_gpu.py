@@ -244,6 +244,47 @@ def test_long_single_sequence_sampled():
         assert rel_l2(g, ref) <= tol, (name, rel_l2(g, ref))
 
 
+def test_maximum_length_sampled():
+    # One sequence of SIGATTN_MAX_LEN = 2^20 tokens at d = 64 (8192 work items per call).
+    B, H, L, d = 1, 1, 1 << 20, 64
+    q, k, v, dout = workloads.make_inputs(B, H, L, d, 64)
+    lens = np.array([L], dtype=np.int32)
+    o, dq, dk, dv = run_gpu(q, k, v, dout, lens)
+    rng = np.random.default_rng(64)
+    row = np.concatenate([[0, L - 1], rng.integers(0, L, 6)])
+    bh = np.zeros_like(row)
+    for name, got, tol in (("o", o, FWD_REL), ("dq", dq, BWD_REL), ("dk", dk, BWD_REL), ("dv", dv, BWD_REL)):
+        ref = oracle.rows(name, q, k, v, dout, lens, bh, row)
+        g = got.reshape(L, d)[row].numpy()
+        assert rel_l2(g, ref) <= tol, (name, rel_l2(g, ref))
+
+
+def test_two_streams_concurrently():
+    # Calls on two streams with their own workspaces may overlap on the GPU; the results are the
+    # same bits as the same calls made one after the other.
+    dev = torch.device("cuda")
+    cases = [(3, 2, 700, 64, [700, 200, 33], 91), (2, 2, 520, 128, [520, 300], 92)]
+    expect = [run_gpu(*workloads.make_inputs(B, H, L, d, seed), lens) for B, H, L, d, lens, seed in cases]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    state = []
+    for (B, H, L, d, lens, seed), st in zip(cases, streams):
+        q, k, v, dout = (t.to(dev) for t in workloads.make_inputs(B, H, L, d, seed))
+        ws = sa.make_workspace(B, H, L, d, dev)
+        outs = [torch.full_like(q, float("nan")) for _ in range(4)]
+        state.append((q, k, v, dout, torch.tensor(lens, dtype=torch.int32, device=dev), ws, outs, st))
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for q, k, v, dout, lens, ws, outs, st in state:
+            sa.sigattn_fwd(q, k, v, outs[0], lens, ws, st)
+            sa.sigattn_bwd_dq(q, k, v, dout, outs[1], lens, ws, st)
+            sa.sigattn_bwd_dkdv(q, k, v, dout, outs[2], outs[3], lens, ws, st)
+    torch.cuda.synchronize()
+    for (q, k, v, dout, lens, ws, outs, st), exp in zip(state, expect):
+        assert sa.sigattn_read_error(ws, st) == (0, 0)
+        for got, ref in zip(outs, exp):
+            assert torch.equal(got.float().cpu(), ref)
+
+
 def test_single_token_sequences_d128():
     # n = 1: bias ln 1 = 0, O_0 = sigma(q.k / sqrt(d)) v
     B, H, L, d = 3, 2, 128, 128
