@@ -228,6 +228,38 @@ def run_reference(args, w):
     return 0
 
 
+def pcie_bandwidth(dev, nbytes: int = 256 << 20, reps: int = 6) -> dict:
+    """Pinned host <-> device copy bandwidth in GB/s: each direction alone, and
+    per direction with both running at once (the bound of a pipelined step)."""
+    import torch
+
+    h_up, h_down = (torch.empty(nbytes, dtype=torch.uint8).pin_memory() for _ in range(2))
+    d_up, d_down = (torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(2))
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def timed(up: bool, down: bool) -> float:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(s_up)
+        s_down.wait_event(e0)
+        for _ in range(reps):
+            if up:
+                with torch.cuda.stream(s_up):
+                    d_up.copy_(h_up, non_blocking=True)
+            if down:
+                with torch.cuda.stream(s_down):
+                    h_down.copy_(d_down, non_blocking=True)
+        s_up.wait_stream(s_down)
+        e1.record(s_up)
+        torch.cuda.synchronize(dev)
+        return reps * nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9
+
+    timed(True, True)  # warm-up
+    out = {"h2d": timed(True, False), "d2h": timed(False, True), "both_per_direction": timed(True, True)}
+    del h_up, h_down, d_up, d_down
+    return out
+
+
 def run_gpu(args, w):
     import torch
 
@@ -415,6 +447,10 @@ def run_gpu(args, w):
     s_in.wait_stream(stream)
     e2e_value = time_e2e(e2e_step_pipelined, s_in, s_out)
     torch.cuda.synchronize(dev)
+    # Bound of the pipelined step: its larger copy direction at the measured
+    # both-directions-at-once PCIe rate, with the compute fully hidden.
+    pcie = pcie_bandwidth(dev)
+    e2e_bound = world * (flops_fwd + flops_bwd) / (max(h2d, d2h) / (pcie["both_per_direction"] * 1e9)) / 1e12
     # The pipelined copies must bring back exactly what the calls wrote.
     for host, devt in zip(outs_h, dev_out):
         if not torch.equal(host, devt.cpu()):
@@ -456,7 +492,9 @@ def run_gpu(args, w):
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps,
                 "schedule": f"{len(rows)} chunks of whole sequences; host-to-device copies, the three calls and "
-                            "device-to-host copies on three streams"},
+                            "device-to-host copies on three streams",
+                "pcie_gbs": pcie, "bound": e2e_bound, "frac_of_bound": e2e_value / e2e_bound,
+                "bound_source": "larger copy direction per step at the measured both-ways pinned copy rate"},
         "e2e_serial": {"value": e2e_serial, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "steps": e2e_steps, "schedule": "copy in, three calls, copy out, one stream"},
         # Device-timed steps only: per call the plan and compute kernels, plus (padded

@@ -35,7 +35,9 @@
 //   XS [0,BN) XdP [BN,2BN) P [2BN,2.5BN) dS [2.5BN,3BN) A1 [3BN,3BN+D) A2 after.
 // Warps: 0-7 epilogue (warps 4g..4g+3 take columns [g BN/2, (g+1) BN/2) of
 // each block), 8 TMA producer (also claims the work items and passes them on
-// through the shared-memory item ring), 9 S issuer (owns TMEM), 10 dP issuer,
+// through the shared-memory item ring; for dQ at D = 64 over padded inputs it
+// also writes the zeros of the rows no item covers, with bulk copies from
+// shared memory while the compute runs), 9 S issuer (owns TMEM), 10 dP issuer,
 // 11 A1 issuer, 12 A2 issuer (dK/dV only). PACKED selects the input layout, as
 // in the forward kernel.
 #include "common.cuh"
@@ -58,7 +60,12 @@ struct BwdCfg {
   static constexpr int OFF_R2 = TILE_R;
   static constexpr int OFF_C1 = 2 * TILE_R;
   static constexpr int OFF_C2 = OFF_C1 + ST1 * TILE_C;
-  static constexpr int SMEM_BYTES = OFF_C2 + ST2 * TILE_C;
+  // dQ at D = 64 over padded inputs: a 16 KB block of zeros in shared memory
+  // from which the producer writes the padded rows of dQ with bulk copies
+  // while the compute runs (at D = 128 the rings leave no room for it).
+  static constexpr int ZBUF = (!KV && D == 64) ? 16384 : 0;
+  static constexpr int OFF_Z = OFF_C2 + ST2 * TILE_C;
+  static constexpr int SMEM_BYTES = OFF_Z + ZBUF;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   static constexpr int TM_XS = 0;
   static constexpr int TM_XDP = BN;
@@ -150,6 +157,14 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     tmem_alloc(&bar.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
+  // Zeros for the producer's bulk fill of padded dQ rows (needs a 16-byte
+  // aligned output; otherwise every unit is left to the tail loop below).
+  const bool bulk_fill = C::ZBUF > 0 && fill_lengths != nullptr && (reinterpret_cast<uintptr_t>(out1) & 15u) == 0;
+  if (bulk_fill) {
+    uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_Z);
+    for (int i = threadIdx.x; i < C::ZBUF / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
   // The plan is written by the kernel before this one in the stream.
   grid_dep_wait();
   tc_fence_before();
@@ -178,6 +193,22 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       bool ok = true;
       uint32_t ist = 0, iph = 0;
       int claimed = -1;
+      // Bulk zero fill: one unit per work item, claimed one item ahead so
+      // that the atomic's latency is not waited for.
+      const long long fill_units = bulk_fill ? static_cast<long long>(B) * H * fill_parts : 0;
+      int fill_u = -1;
+      auto issue_fill = [&]() {
+        if constexpr (C::ZBUF > 0) {
+          if (fill_u >= 0 && fill_u < fill_units) {
+            const FillRange f = zero_fill_range(fill_lengths, H, L, D, C::BM, fill_parts, fill_u);
+            uint8_t* g = reinterpret_cast<uint8_t*>(out1 + f.base);
+            constexpr long long kPiece = C::ZBUF / 16;  // 16-byte chunks per bulk copy
+            for (long long c = f.begin; c < f.end; c += kPiece)
+              bulk_store(g + c * 16, sbase + C::OFF_Z, static_cast<uint32_t>(min(kPiece, f.end - c) * 16));
+            bulk_commit();
+          }
+        }
+      };
       while (ok) {
         const Item item = next_item(ws, claimed, count);
         if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, ws, 200))) break;
@@ -185,6 +216,10 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         const int n = item.n;
         const int hd = PACKED ? item.bh % H : 0;
         const int nb = ceil_div(n, C::BN);
+        if (fill_units > 0 && fill_u < fill_units) {
+          issue_fill();
+          fill_u = atomicAdd(ws + kHdrFill, 1);
+        }
         if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, ws, 201))) break;
         mbar_arrive_expect_tx(&bar.r_full, 2 * C::TILE_R);
         for (int c = 0; c < D / 64; ++c) {
@@ -212,6 +247,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           c2_last[s2] = static_cast<int>(p2);
           if (++s2 == C::ST2) { s2 = 0; p2 ^= 1; }
         }
+      }
+      // The last unit claimed, then every bulk copy must have landed before
+      // the shared-memory zeros go away with the CTA.
+      if (fill_units > 0) {
+        issue_fill();
+        bulk_wait_all();
       }
       if (!ok) {  // aborting: let the copies in flight land before the CTA exits
         int never = 0;
@@ -496,18 +537,18 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     }
   }
 
-  // dQ over padded inputs: the rows no item covers are zeroed here, in the
-  // kernel's tail. Each warp joins once its role is done and claims fill units
-  // from the workspace counter, so the CTAs that run out of items first do
-  // most of it.
-  if (fill_lengths != nullptr) {
+  // dQ over padded inputs: the fill units the producer did not take (all of
+  // them at D = 128, which has no room for the zeros in shared memory) are
+  // zeroed here, in the kernel's tail. Each warp joins once its role is done
+  // and claims units from the same workspace counter.
+  if (!KV && fill_lengths != nullptr) {
     const long long units = static_cast<long long>(B) * H * fill_parts;
     while (true) {
       int u = 0;
       if (lane == 0) u = atomicAdd(ws + kHdrFill, 1);
       u = __shfl_sync(0xffffffffu, u, 0);
       if (u >= units) break;
-      zero_fill_unit(fill_lengths, H, L, D, C::BM, fill_parts, u, lane, out1, nullptr);
+      zero_fill_range_warp(zero_fill_range(fill_lengths, H, L, D, C::BM, fill_parts, u), lane, out1);
     }
   }
 

@@ -171,6 +171,35 @@ __device__ __forceinline__ void zero_fill_unit(const int* lengths, int H, int L,
   }
 }
 
+// The same rows cut into `parts` consecutive shares instead (the dQ kernel's
+// fill, whose units go either to bulk copies or to warps): unit u covers the
+// 16-byte chunks [begin, end) counted from element `base` of the output.
+struct FillRange {
+  size_t base;
+  long long begin, end;
+};
+
+__device__ __forceinline__ FillRange zero_fill_range(const int* lengths, int H, int L, int d, int rows, int parts,
+                                                     long long u) {
+  const int slice = static_cast<int>(u / parts);
+  const int part = static_cast<int>(u % parts);
+  const int n = load_len(lengths, slice / H, L);
+  const int cover = min(L, ceil_div(n, rows) * rows);
+  const long long nchunks = static_cast<long long>(L - cover) * (d / 8);
+  const long long share = (nchunks + parts - 1) / parts;
+  FillRange f;
+  f.base = (static_cast<size_t>(slice) * L + cover) * d;
+  f.begin = min(nchunks, part * share);
+  f.end = min(nchunks, f.begin + share);
+  return f;
+}
+
+// One warp writes the zeros of a consecutive-share unit.
+__device__ __forceinline__ void zero_fill_range_warp(const FillRange& f, int lane, __nv_bfloat16* out) {
+  uint4* p = reinterpret_cast<uint4*>(out + f.base);
+  for (long long c = f.begin + lane; c < f.end; c += 32) p[c] = make_uint4(0, 0, 0, 0);
+}
+
 // Shares per slice for the zero fill: enough units to spread over the SMs.
 inline int zero_fill_parts(long long slices, int num_sms) {
   return static_cast<int>(std::max<long long>(1, std::min<long long>(64, (4LL * num_sms + slices - 1) / slices)));

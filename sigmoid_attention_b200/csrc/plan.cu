@@ -16,8 +16,10 @@
 //     fill_kernel, a one-warp-per-CTA kernel launched with a programmatic edge,
 //     so that it runs on the registers and warps the persistent compute CTA
 //     leaves free and its HBM writes overlap the compute-bound kernel; the dQ
-//     kernel zeroes its own in its tail (each warp, once its role is done,
-//     claims fill units from a counter in the workspace header).
+//     kernel zeroes its own: at d = 64 its producer issues bulk copies from a
+//     block of zeros in shared memory, one fill unit per work item, and in its
+//     tail each warp, once its role is done, claims the units left from the
+//     same counter in the workspace header.
 #include <algorithm>
 #include <numeric>
 #include <vector>
