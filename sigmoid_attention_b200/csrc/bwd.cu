@@ -157,8 +157,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     tmem_alloc(&bar.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  // Zeros for the producer's bulk fill of padded dQ rows (needs a 16-byte
-  // aligned output; otherwise every unit is left to the tail loop below).
+  // Zeros for the producer's bulk fill of padded dQ rows. Bulk copies need
+  // 16-byte aligned addresses; the host already rejects outputs that are not,
+  // and the check here keeps the rule next to the copies.
   const bool bulk_fill = C::ZBUF > 0 && fill_lengths != nullptr && (reinterpret_cast<uintptr_t>(out1) & 15u) == 0;
   if (bulk_fill) {
     uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_Z);
