@@ -27,11 +27,10 @@
  *    bias has no gradient. There is no causal mask.
  *  - Arithmetic: bf16 operands, fp32 accumulation, P (and dS) rounded to bf16
  *    before the second matrix product, outputs rounded to nearest bf16. sigma
- *    is computed as 1/2 + tanh(x/2)/2 with the hardware tanh (one MUFU
- *    operation per score) when Lmax <= 65536; above that the bias -ln(n) puts
- *    most weights below 1e-5, where that route's absolute error becomes a
- *    relative error of percent size, so calls with a larger Lmax (max_seqlen
- *    for the packed calls) use 1/(1 + 2^(-x log2 e)) (two MUFU operations).
+ *    takes one hardware exp2 per score: with u = e^-|x|, sigma(x) = u r(u)
+ *    for x < 0 and r(u) for x >= 0, where r is a polynomial for 1/(1+u) of
+ *    relative error <= 8e-4 (about 1e-7 for the tail weights near 1/n that
+ *    the bias -ln n makes typical); see sigattn_eval_sigmoid.
  *  - workspace: caller-owned device memory of at least
  *    sigattn_workspace_size(B, H, Lmax, d) bytes, 16-byte aligned. Each call
  *    writes its work list there; calls that may run concurrently (different
@@ -177,9 +176,13 @@ SIGATTN_API int sigattn_plan_host(const int32_t* lengths_host, int B, int H, int
  *    (cudaGetSymbolAddress); make that first call before any stream capture.
  *  - Every call, on every stream, shares the one array: calls that overlap
  *    on the GPU race. Each call clears the array's status words first.
- *  - status_out: optional device int32; if not NULL, receives (in stream
- *    order) this call's device-side status: 0, SIGATTN_ERR_INVALID_ARG for an
- *    out-of-range length, or SIGATTN_ERR_TIMEOUT. */
+ *  - status_out: optional device int32 (4-byte aligned); if not NULL, it
+ *    receives (in stream order) this call's device-side status: 0,
+ *    SIGATTN_ERR_INVALID_ARG for an out-of-range length, or
+ *    SIGATTN_ERR_TIMEOUT.
+ *  - Argument errors (the checks of sigattn_fwd, a misaligned status_out, a
+ *    size beyond the array) are returned before anything is enqueued and
+ *    leave the array untouched. */
 SIGATTN_API int sigattn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, const int32_t* lengths,
                                     int B, int H, int Lmax, int d, int32_t* status_out, void* stream);
 
@@ -194,6 +197,18 @@ SIGATTN_API const char* sigattn_last_error(void);
  * does, and returns normally (the context stays usable). Needs only the
  * 256-byte header of a workspace. */
 SIGATTN_API int sigattn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int limit_us, void* stream);
+
+/* Diagnostic: the attention weight of raw scores exactly as the compute
+ * kernels evaluate it, P = sigma(s / sqrt(d) - ln n) (sec. 2A: the sigmoid of
+ * the scaled score plus the bias b = -ln n), and its derivative
+ * P (1 - P) (sec. 2B) as the backward kernels use it. scores, p and slope are
+ * device float arrays of `count` elements (4-byte aligned); d is 64 or 128,
+ * 1 <= n <= SIGATTN_MAX_LEN. The kernels form x = s / sqrt(d) - ln n and
+ * take sigma from one hardware exp2 of -|x| log2(e) and a polynomial for
+ * 1/(1 + e^-|x|); this entry point lets a test measure that form's error
+ * against the exact function on any set of scores. Stream-ordered, no sync. */
+SIGATTN_API int sigattn_eval_sigmoid(const float* scores, float* p, float* slope, int count, int d, int n,
+                                     void* stream);
 
 /* Synchronise `stream`, read the workspace's sticky error word, clear it and
  * return it (SIGATTN_OK if no kernel reported a problem). If `site` is not

@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "SigattnError", "library", "library_path", "sigattn_version", "sigattn_status_str", "sigattn_block_rows",
     "sigattn_workspace_size", "sigattn_fwd", "sigattn_fwd_noalloc", "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
-    "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
+    "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "sigattn_eval_sigmoid", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
     "sigattn_fwd_varlen", "sigattn_bwd_dq_varlen", "sigattn_bwd_dkdv_varlen",
     "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
     "SigmoidAttentionVarlenFunction", "sigmoid_attention_varlen",
@@ -87,6 +87,8 @@ def library():
         lib.sigattn_selftest_wait_timeout.argtypes = [_vp, _sz, _i, _vp]
         lib.sigattn_last_error.restype = ctypes.c_char_p
         lib.sigattn_last_error.argtypes = []
+        lib.sigattn_eval_sigmoid.restype = _i
+        lib.sigattn_eval_sigmoid.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp]
         lib.sigattn_read_error.restype = _i
         lib.sigattn_read_error.argtypes = [_vp, ctypes.POINTER(_i), _vp]
         _lib = lib
@@ -243,6 +245,16 @@ def sigattn_selftest_wait_timeout(workspace, limit_us: int = 20000, stream=None)
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), int(limit_us), _stream_ptr(stream)))
 
 
+def sigattn_eval_sigmoid(scores, d: int, n: int, stream=None):
+    """(P, slope) of float32 CUDA scores as the kernels compute them:
+    P = sigma(s / sqrt(d) - ln n), slope = P (1 - P)."""
+    p, slope = torch.empty_like(scores), torch.empty_like(scores)
+    _check("sigattn_eval_sigmoid", library().sigattn_eval_sigmoid(
+        _dev(scores, "scores", torch.float32), _dev(p, "p", torch.float32), _dev(slope, "slope", torch.float32),
+        scores.numel(), int(d), int(n), _stream_ptr(stream)))
+    return p, slope
+
+
 def sigattn_last_error() -> str:
     return library().sigattn_last_error().decode()
 
@@ -277,27 +289,48 @@ def backward(q, k, v, dout, lengths, workspace=None, stream=None):
     return dq, dk, dv
 
 
+def _check_device_status(fn: str, workspace, check: bool) -> None:
+    """With ``check`` (or SIGATTN_CHECK=1 in the environment), synchronise and
+    raise if a kernel flagged an out-of-range length or an expired wait in the
+    workspace's sticky status word (otherwise such a sequence's outputs are
+    zeros and nothing is raised)."""
+    if not (check or os.environ.get("SIGATTN_CHECK", "0") == "1"):
+        return
+    st, site = sigattn_read_error(workspace)
+    if st != 0:
+        err = SigattnError(fn, st)
+        err.args = (f"{err.args[0]} (device status, site {site})",)
+        raise err
+
+
 class SigmoidAttentionFunction(torch.autograd.Function):
     """Autograd wrapper: forward with ``sigattn_fwd``, backward with the two
     backward calls (a drop-in for softmax attention over padded batches)."""
 
     @staticmethod
-    def forward(ctx, q, k, v, lengths):
+    def forward(ctx, q, k, v, lengths, check=False):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         ws = make_workspace(*_dims(q), q.device)
         o = forward(q, k, v, lengths, ws)
+        _check_device_status("sigattn_fwd", ws, check)
         ctx.save_for_backward(q, k, v, lengths, ws)
+        ctx.check = check
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, lengths, ws = ctx.saved_tensors
         dq, dk, dv = backward(q, k, v, do.contiguous(), lengths, ws)
-        return dq, dk, dv, None
+        _check_device_status("sigattn_bwd", ws, ctx.check)
+        return dq, dk, dv, None, None
 
 
-def sigmoid_attention(q, k, v, lengths) -> torch.Tensor:
-    return SigmoidAttentionFunction.apply(q, k, v, lengths)
+def sigmoid_attention(q, k, v, lengths, check: bool = False) -> torch.Tensor:
+    """O = sigma(q k^T / sqrt(d) - ln n) v over padded [B, H, Lmax, d] bf16
+    tensors, differentiable in q, k, v. ``check=True`` synchronises after the
+    forward and the backward calls and raises SigattnError when a kernel
+    reported a problem (an out-of-range length, an expired wait)."""
+    return SigmoidAttentionFunction.apply(q, k, v, lengths, check)
 
 
 class SigmoidAttentionVarlenFunction(torch.autograd.Function):
@@ -305,14 +338,16 @@ class SigmoidAttentionVarlenFunction(torch.autograd.Function):
     with sequences back to back as given by cu_seqlens (int32 [B + 1])."""
 
     @staticmethod
-    def forward(ctx, q, k, v, cu_seqlens, max_seqlen):
+    def forward(ctx, q, k, v, cu_seqlens, max_seqlen, check=False):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         _, H, d = _packed_dims(q)
         ws = make_workspace(cu_seqlens.numel() - 1, H, max_seqlen, d, q.device)
         o = torch.empty_like(q)
         sigattn_fwd_varlen(q, k, v, o, cu_seqlens, max_seqlen, ws)
+        _check_device_status("sigattn_fwd_varlen", ws, check)
         ctx.save_for_backward(q, k, v, cu_seqlens, ws)
         ctx.max_seqlen = max_seqlen
+        ctx.check = check
         return o
 
     @staticmethod
@@ -322,8 +357,11 @@ class SigmoidAttentionVarlenFunction(torch.autograd.Function):
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         sigattn_bwd_dq_varlen(q, k, v, do, dq, cu_seqlens, ctx.max_seqlen, ws)
         sigattn_bwd_dkdv_varlen(q, k, v, do, dk, dv, cu_seqlens, ctx.max_seqlen, ws)
-        return dq, dk, dv, None, None
+        _check_device_status("sigattn_bwd_varlen", ws, ctx.check)
+        return dq, dk, dv, None, None, None
 
 
-def sigmoid_attention_varlen(q, k, v, cu_seqlens, max_seqlen: int) -> torch.Tensor:
-    return SigmoidAttentionVarlenFunction.apply(q, k, v, cu_seqlens, int(max_seqlen))
+def sigmoid_attention_varlen(q, k, v, cu_seqlens, max_seqlen: int, check: bool = False) -> torch.Tensor:
+    """The packed-layout counterpart of ``sigmoid_attention`` ([total, H, d]
+    tensors, int32 cu_seqlens [B + 1]); ``check`` as there."""
+    return SigmoidAttentionVarlenFunction.apply(q, k, v, cu_seqlens, int(max_seqlen), check)

@@ -18,6 +18,8 @@ cudaError_t launch_fill(const int* lengths, int B, int H, int L, int d, int kind
                         int num_sms, cudaStream_t stream);
 int plan_host(const int* lengths, int B, int H, int L, int kind, int* out, int cap);
 cudaError_t launch_selftest_timeout(int* ws, unsigned long long limit_ns, cudaStream_t stream);
+cudaError_t launch_eval_sigmoid(const float* s, float* p, float* slope, int count, int d, int n, int num_sms,
+                                cudaStream_t stream);
 cudaError_t launch_fwd(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        void* o, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_dq(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
@@ -59,6 +61,7 @@ struct DeviceInfo {
 bool device_info(DeviceInfo* out) {
   static DeviceInfo cache[64];
   static bool have[64] = {};
+  static std::once_flag once[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   // A thread that has not used this library's CUDA runtime yet (for example
@@ -69,15 +72,17 @@ bool device_info(DeviceInfo* out) {
     if (cudaSetDevice(dev) != cudaSuccess) return false;
     ready_for = dev;
   }
-  if (!have[dev]) {
+  // Queried once per device (safely across host threads).
+  std::call_once(once[dev], [dev] {
     int major = 0, minor = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
-    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return;
     cache[dev].num_sms = sms;
     cache[dev].supported = (major == 10 && minor == 0);
     have[dev] = true;
-  }
+  });
+  if (!have[dev]) return false;
   *out = cache[dev];
   return true;
 }
@@ -167,6 +172,31 @@ int check_call(int B, int H, int L, int d, const int32_t* lengths, const void* w
 }
 
 }  // namespace
+
+namespace sigattn {
+
+// The host checks of a padded-layout forward call that do not involve a
+// workspace: sizes, the lengths pointer, 16-byte alignment of q, k, v, o and
+// the device's architecture (for entry points that bring their own scratch).
+int check_fwd_inputs(const void* q, const void* k, const void* v, const void* o, const int32_t* lengths, int B,
+                     int H, int L, int d) {
+  int st = check_sizes(B, H, L, d);
+  if (st != SIGATTN_OK) return st;
+  if (lengths == nullptr || (reinterpret_cast<uintptr_t>(lengths) & 3u) != 0) return SIGATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SIGATTN_ERR_INVALID_ARG;
+  DeviceInfo info;
+  if (!device_info(&info)) {
+    const cudaError_t e = cudaGetLastError();
+    return cuda_status(e != cudaSuccess ? e : cudaErrorUnknown);
+  }
+  return info.supported ? SIGATTN_OK : SIGATTN_ERR_UNSUPPORTED;
+}
+
+// SIGATTN_OK for cudaSuccess; otherwise records the error's text for
+// sigattn_last_error and returns SIGATTN_ERR_CUDA.
+int report_cuda(cudaError_t e) { return cuda_status(e); }
+
+}  // namespace sigattn
 
 extern "C" {
 
@@ -346,6 +376,18 @@ int sigattn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int l
   return cuda_status(launch_selftest_timeout(static_cast<int*>(workspace),
                                              static_cast<unsigned long long>(limit_us) * 1000ull,
                                              static_cast<cudaStream_t>(stream)));
+}
+
+int sigattn_eval_sigmoid(const float* scores, float* p, float* slope, int count, int d, int n, void* stream) {
+  if (d != 64 && d != 128) return SIGATTN_ERR_UNSUPPORTED;
+  if (count < 0 || n < 1 || n > kMaxLen) return SIGATTN_ERR_INVALID_ARG;
+  if (count == 0) return SIGATTN_OK;
+  const auto aligned4 = [](const void* ptr) { return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; };
+  if (!aligned4(scores) || !aligned4(p) || !aligned4(slope)) return SIGATTN_ERR_INVALID_ARG;
+  DeviceInfo info;
+  if (!device_info(&info)) return cuda_status(cudaErrorUnknown);
+  if (!info.supported) return SIGATTN_ERR_UNSUPPORTED;
+  return cuda_status(launch_eval_sigmoid(scores, p, slope, count, d, n, info.num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 int sigattn_read_error(void* workspace, int* site, void* stream) {

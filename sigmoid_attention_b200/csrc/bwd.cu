@@ -101,8 +101,7 @@ struct BwdBarriers {
   int abort;
 };
 
-// ACC: the accurate sigmoid route (calls whose Lmax exceeds kAccurateSigmoidLen).
-template <int D, bool KV, bool PACKED, bool ACC>
+template <int D, bool KV, bool PACKED>
 __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_r1, const __grid_constant__ CUtensorMap tm_r2,
                const __grid_constant__ CUtensorMap tm_c1, const __grid_constant__ CUtensorMap tm_c2,
@@ -384,8 +383,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     const uint32_t tXDP0 = tmem + lane_off + C::TM_XDP + g * CPW * 32;
     const uint32_t tXDP1 = tmem + lane_off + C::TM_XDP1 + g * CPW * 32;
     constexpr float scale = Scale<D>::value;
-    constexpr float half_scale = 0.5f * scale;
-    constexpr float neg_scale_l2e = -scale * 1.4426950408889634f;
+    const uint64_t scale_l2e2 = f2_splat(scale * kLog2e);
     uint32_t s_ph = 0, free_ph = 0, aph = 0, xb = 0;
     uint32_t dp_ph[2] = {0, 0};
     bool ok = true;
@@ -398,11 +396,13 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       if (item.n < 0) break;
       const int n = item.n;
       const int nb = ceil_div(n, C::BN);
-      const float half_bias = -0.5f * __logf(static_cast<float>(n));
-      const float neg_bias_l2e = __log2f(static_cast<float>(n));  // -bias * log2(e)
+      const uint64_t neg_log2n2 = f2_splat(-__log2f(static_cast<float>(n)));  // bias * log2(e)
       for (int j = 0; j < nb; ++j) {
-        // ---- S -> P (fp32 kept in registers for dS), bf16 P for dV
-        float p[CPW][32];
+        // ---- S -> sigma'(x) = P (1 - P) kept in registers for dS, and (dK/dV)
+        // bf16 P for dV, stored chunk by chunk as it is computed (the P region
+        // is free once the previous block's dV products have read it). Padded
+        // columns get P = sigma' = 0.
+        uint64_t sp[CPW][16];  // sigma' of column pairs (2e, 2e + 1)
         {
           uint32_t sv[CPW][32];
           if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, ws, 221))) break;
@@ -415,33 +415,36 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.xs_read);
+          if (KV) {
+            if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
+            tc_fence_after();
+          }
           const int valid = n - (j * C::BN + g * CPW * 32);  // columns < valid are real tokens
-          auto chunks_p = [&](auto accurate) {
-            constexpr bool kAcc = decltype(accurate)::value;
-#pragma unroll
-            for (int c = 0; c < CPW; ++c)
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const float pe =
-                    sigmoid_of<kAcc>(__uint_as_float(sv[c][e]), half_scale, half_bias, neg_scale_l2e, neg_bias_l2e);
-                p[c][e] = (valid >= CPW * 32 || 32 * c + e < valid) ? pe : 0.f;
-              }
-          };
-          chunks_p(std::integral_constant<bool, ACC>{});
-        }
-        if (KV) {
-          if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
-          tc_fence_after();
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
             uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(p[c][2 * e], p[c][2 * e + 1]);
-            tmem_st16(tmem + lane_off + C::TM_P + (g * CPW + c) * 16, pk);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar.p_full[g * CPW + c]);
+            for (int e = 0; e < 16; ++e) {
+              uint64_t slope;
+              const uint64_t pp = sigmoid2<true>(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1]),
+                                                 scale_l2e2, neg_log2n2, &slope);
+              if (valid < CPW * 32) {
+                const float2 p = f2_unpack(pp), d = f2_unpack(slope);
+                const bool v0 = 32 * c + 2 * e < valid, v1 = 32 * c + 2 * e + 1 < valid;
+                pk[e] = pack_bf16x2(v0 ? p.x : 0.f, v1 ? p.y : 0.f);
+                sp[c][e] = f2_pack(v0 ? d.x : 0.f, v1 ? d.y : 0.f);
+              } else {
+                pk[e] = pack_bf16x2_pair(pp);
+                sp[c][e] = slope;
+              }
+            }
+            if (KV) {
+              tmem_st16(tmem + lane_off + C::TM_P + (g * CPW + c) * 16, pk);
+              tmem_st_wait();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bar.p_full[g * CPW + c]);
+            }
           }
         }
         // ---- dP -> dS = dP P (1 - P), bf16 dS for dQ / dK. The dK/dV kernel
@@ -477,15 +480,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
               if (lane == 0) mbar_arrive(xdp_read);
             }
           }
-          uint32_t pk[16];
+          uint32_t dk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float q0 = p[c][2 * e], q1 = p[c][2 * e + 1];
-            const float ds0 = __uint_as_float(dpc[2 * e]) * (q0 - q0 * q0);
-            const float ds1 = __uint_as_float(dpc[2 * e + 1]) * (q1 - q1 * q1);
-            pk[e] = pack_bf16x2(ds0, ds1);
-          }
-          tmem_st16(tmem + lane_off + C::TM_DS + (g * CPW + c) * 16, pk);
+          for (int e = 0; e < 16; ++e)
+            dk[e] = pack_bf16x2_pair(f2_mul(f2_pack(__uint_as_float(dpc[2 * e]), __uint_as_float(dpc[2 * e + 1])),
+                                            sp[c][e]));
+          tmem_st16(tmem + lane_off + C::TM_DS + (g * CPW + c) * 16, dk);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
@@ -561,38 +561,23 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   }
 }
 
-template <int D, bool KV, bool PACKED, bool ACC>
+template <int D, bool KV, bool PACKED>
 cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
                             const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
                             const int* fill_lengths, cudaStream_t stream) {
   using C = BwdCfg<D, KV>;
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED, ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static PerDeviceOnce attr;
+  const cudaError_t e = attr.run([] {
+    return cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_ALLOC);
+  });
+  if (e != cudaSuccess) return e;
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kBwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
   const int parts = zero_fill_parts(static_cast<long long>(B) * H, num_sms);
-  return launch_programmatic(bwd_kernel<D, KV, PACKED, ACC>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2,
+  return launch_programmatic(bwd_kernel<D, KV, PACKED>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2,
                              c1, c2, static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), ws, H, L,
                              fill_lengths, B, parts);
-}
-
-template <int D, bool KV, bool PACKED>
-cudaError_t launch_bwd_acc(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1, const CUtensorMap& c2,
-                           void* out1, void* out2, int* ws, int B, int H, int L, int num_sms, const int* fill_lengths,
-                           cudaStream_t stream) {
-  // No sequence is longer than L, so L decides the sigmoid route for the call.
-  if (L > kAccurateSigmoidLen)
-    return launch_bwd_impl<D, KV, PACKED, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths,
-                                                stream);
-  return launch_bwd_impl<D, KV, PACKED, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths,
-                                               stream);
 }
 
 template <bool KV>
@@ -601,12 +586,12 @@ cudaError_t launch_bwd(int d, bool packed, const CUtensorMap& r1, const CUtensor
                        const int* fill_lengths, cudaStream_t stream) {
   if (packed) {
     if (d == 64)
-      return launch_bwd_acc<64, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
-    return launch_bwd_acc<128, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
+      return launch_bwd_impl<64, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
+    return launch_bwd_impl<128, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
   }
   if (d == 64)
-    return launch_bwd_acc<64, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
-  return launch_bwd_acc<128, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
+    return launch_bwd_impl<64, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
+  return launch_bwd_impl<128, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
 }
 
 // fill_lengths: the padded layout's lengths, so that the dQ kernel zeroes the

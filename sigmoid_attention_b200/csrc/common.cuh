@@ -4,6 +4,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 #include <type_traits>
 #include <utility>
 #include <cuda_bf16.h>
@@ -142,13 +143,92 @@ struct Scale<128> {
   static constexpr float value = 0.08838834764831845f;
 };
 
-// sigma(s * scale + bias) for one score, written as 1/2 + tanh(x/2)/2 with the
-// hardware tanh ("a hardware-optimised tanh approximation for the sigmoid",
-// Better Models, Faster Training, sec. 2C). half_scale = scale/2 and
-// half_bias = bias/2 are folded into one FMA.
-__device__ __forceinline__ float sigmoid_from_score(float s, float half_scale, float half_bias) {
-  const float t = tanh_approx(fmaf(s, half_scale, half_bias));
-  return fmaf(t, 0.5f, 0.5f);
+// The sigmoid of a score, with one MUFU operation. For a score s of sequence
+// length n the argument is x = s / sqrt(d) - ln n (Better Models, Faster
+// Training: Sigmoid Attention for single-cell Foundation Models, sec. 2A); the
+// kernels form y = x log2(e) = s * scale_l2e + neg_log2n in one FMA and take
+//
+//   u = 2^(-|y|) = e^(-|x|)              (ex2.approx, relative error ~1e-7)
+//   r = 1 - u + kR2 u^2 + kR3 u^3 + kR4 u^4  ~  1 / (1 + u) on [0, 1]
+//   q = u r ~ sigma(-|x|),   sigma(x) = q for x < 0, r for x >= 0,
+//   sigma'(x) = sigma(x) sigma(-x) = q r.
+//
+// The polynomial keeps r(0) = 1 and r'(0) = -1 exactly, so the weights of the
+// far tail (the usual case: the bias puts typical weights near 1/n) carry a
+// relative error of ~1e-6, and r(1) = 1/2, so sigma(0) = 1/2 and sigma'(0) =
+// 1/4; a minimax fit of the other coefficients bounds the relative error of
+// sigma by 9e-4 over the whole line (largest near |x| = 1.5), below the bf16
+// rounding that P undergoes next.
+//
+// The pages' kernel takes sigma from the hardware tanh, 1/2 + tanh(x/2)/2
+// (sec. 2C). Measured on B200, that form's error is a few 1e-6 in absolute
+// terms, which near 1/n is a relative error of up to 1 % (x in [-12, -8]) and
+// which drops every weight below ~1e-7 to zero; with all weights of a row near
+// 1/n it shifts O by the same relative amount. The form here costs the same
+// single MUFU operation per score; its FMAs run two scores at a time on the
+// packed fp32x2 pipe of sm_100, so it adds about three issue slots per score.
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kR2 = 0.9339003266f;
+constexpr float kR3 = -0.6298789201f;
+constexpr float kR4 = 0.1959785935f;
+
+// Two fp32 values in one 64-bit register (low half = first), for the packed
+// fp32x2 arithmetic of sm_100 (one instruction per two values).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__host__ __device__ constexpr uint64_t f2_splat_bits(uint32_t bits) {
+  return (static_cast<uint64_t>(bits) << 32) | bits;
+}
+__device__ __forceinline__ uint64_t f2_splat(float x) { return f2_splat_bits(__float_as_uint(x)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// sigma of two scores (a, b) at once, as an fp32 pair; with `slope` also
+// sigma' of both. scale_l2e2 and neg_log2n2 are splat pairs of
+// scale * log2(e) and -log2(n).
+template <bool SLOPE>
+__device__ __forceinline__ uint64_t sigmoid2(float a, float b, uint64_t scale_l2e2, uint64_t neg_log2n2,
+                                             uint64_t* slope) {
+  const float2 y = f2_unpack(f2_fma(f2_pack(a, b), scale_l2e2, neg_log2n2));
+  const uint64_t u = f2_pack(ex2_approx(-fabsf(y.x)), ex2_approx(-fabsf(y.y)));
+  uint64_t r = f2_fma(f2_splat(kR4), u, f2_splat(kR3));
+  r = f2_fma(r, u, f2_splat(kR2));
+  r = f2_fma(r, u, f2_splat(-1.0f));
+  r = f2_fma(r, u, f2_splat(1.0f));
+  const uint64_t q = f2_mul(u, r);
+  if (SLOPE) *slope = f2_mul(q, r);
+  const float2 qq = f2_unpack(q), rr = f2_unpack(r);
+  return f2_pack(y.x < 0.0f ? qq.x : rr.x, y.y < 0.0f ? qq.y : rr.y);
+}
+
+// sigma of one score (the diagnostic entry point; the kernels use sigmoid2).
+__device__ __forceinline__ float sigmoid_score(float s, float scale_l2e, float neg_log2n, float* slope) {
+  uint64_t sl = 0;
+  const float2 p = f2_unpack(sigmoid2<true>(s, s, f2_splat(scale_l2e), f2_splat(neg_log2n), &sl));
+  *slope = f2_unpack(sl).x;
+  return p.x;
+}
+
+// Pack an fp32 pair to a bf16x2 word (round to nearest even; first value low).
+__device__ __forceinline__ uint32_t pack_bf16x2_pair(uint64_t v) {
+  const float2 f = f2_unpack(v);
+  return pack_bf16x2(f.x, f.y);
 }
 
 // Zero one unit of the output rows that no work item covers: rows
@@ -225,27 +305,6 @@ __device__ __forceinline__ void store_row64B(void* dst, const uint32_t (&w)[16])
   }
 }
 
-// sigma for long sequences. The bias -ln(n) puts the typical weight near 1/n;
-// for n beyond kAccurateSigmoidLen the tanh route computes those weights just
-// above tanh = -1, where the hardware tanh's absolute error becomes a relative
-// error of several percent (measured: O rel-L2 1.1e-2 at n = 2^20). There
-// sigma = 1 / (1 + 2^(-x log2 e)) is used instead: two MUFU operations (ex2,
-// rcp) per score, relative error ~1e-6 everywhere. neg_scale_l2e = -scale *
-// log2(e), neg_bias_l2e = ln(n) * log2(e) = log2(n).
-constexpr int kAccurateSigmoidLen = 65536;
-
-__device__ __forceinline__ float sigmoid_accurate(float s, float neg_scale_l2e, float neg_bias_l2e) {
-  return rcp_approx(1.0f + ex2_approx(fmaf(s, neg_scale_l2e, neg_bias_l2e)));
-}
-
-// ACCURATE (a kernel template parameter, chosen per call from Lmax) selects
-// sigmoid_accurate.
-template <bool ACCURATE>
-__device__ __forceinline__ float sigmoid_of(float s, float half_scale, float half_bias, float neg_scale_l2e,
-                                            float neg_bias_l2e) {
-  return ACCURATE ? sigmoid_accurate(s, neg_scale_l2e, neg_bias_l2e) : sigmoid_from_score(s, half_scale, half_bias);
-}
-
 // Convert 32 fp32 accumulator values (times `mul`) to bf16 and store them.
 __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul) {
   uint32_t w[16];
@@ -261,6 +320,23 @@ __device__ __forceinline__ void store_zero32(__nv_bfloat16* dst) {
   for (int e = 0; e < 16; ++e) w[e] = 0u;
   store_row64B(dst, w);
 }
+
+// A set-up step (a kernel attribute) run once per device, safely across host
+// threads: the first caller on a device runs it, later callers get its result.
+struct PerDeviceOnce {
+  static constexpr int kDevices = 64;
+  std::once_flag flag[kDevices];
+  cudaError_t err[kDevices] = {};
+  template <typename F>
+  cudaError_t run(F&& setup) {
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kDevices) return cudaErrorInvalidDevice;
+    std::call_once(flag[dev], [&] { err[dev] = setup(); });
+    return err[dev];
+  }
+};
 
 // Launch `kernel` so that it may start while the previous kernel in `stream` is
 // still running (programmatic stream serialization). The kernel calls

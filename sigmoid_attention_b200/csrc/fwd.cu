@@ -81,8 +81,7 @@ struct FwdBarriers {
   int abort;
 };
 
-// ACC: the accurate sigmoid route (calls whose Lmax exceeds kAccurateSigmoidLen).
-template <int D, bool PACKED, bool ACC>
+template <int D, bool PACKED>
 __global__ void __launch_bounds__((16 + 3) * 32, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
@@ -348,8 +347,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     const int r = ((warp & 3) << 5) + lane;        // row within a tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
     const int ot = c >> 1, oc = c & 1;
-    constexpr float half_scale = 0.5f * Scale<D>::value;
-    constexpr float neg_scale_l2e = -Scale<D>::value * 1.4426950408889634f;
+    const uint64_t scale_l2e2 = f2_splat(Scale<D>::value * kLog2e);
     uint32_t sph[2] = {0, 0}, oph[2] = {0, 0}, pvph[2] = {0, 0};
     bool pv_pending[2] = {false, false};  // a P of the tile was written whose PV has not been awaited
     bool ok = true;
@@ -364,8 +362,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       const int row_base = item.blk * (C::BM * C::NQ);
       const int ntiles = (row_base + C::BM < n) ? 2 : 1;
       const int nkb = ceil_div(n, C::BN);
-      const float half_bias = -0.5f * __logf(static_cast<float>(n));
-      const float neg_bias_l2e = __log2f(static_cast<float>(n));  // -bias * log2(e)
+      const uint64_t neg_log2n2 = f2_splat(-__log2f(static_cast<float>(n)));  // bias * log2(e)
       for (int j = 0; ok && j < nkb; ++j) {
         const int valid = n - (j * C::BN + 32 * c);  // columns < valid are real keys
         for (int t = 0; t < ntiles; ++t) {
@@ -378,21 +375,17 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.s_read[t]);
           uint32_t pk[16];
-          auto chunk_p = [&](auto accurate) {
-            constexpr bool kAcc = decltype(accurate)::value;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float p0 = sigmoid_of<kAcc>(__uint_as_float(a[2 * e]), half_scale, half_bias, neg_scale_l2e, neg_bias_l2e);
-              float p1 =
-                  sigmoid_of<kAcc>(__uint_as_float(a[2 * e + 1]), half_scale, half_bias, neg_scale_l2e, neg_bias_l2e);
-              if (valid < 32) {
-                p0 = (2 * e < valid) ? p0 : 0.f;
-                p1 = (2 * e + 1 < valid) ? p1 : 0.f;
-              }
-              pk[e] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t pp = sigmoid2<false>(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]), scale_l2e2,
+                                                neg_log2n2, nullptr);
+            if (valid < 32) {
+              const float2 p = f2_unpack(pp);
+              pk[e] = pack_bf16x2((2 * e < valid) ? p.x : 0.f, (2 * e + 1 < valid) ? p.y : 0.f);
+            } else {
+              pk[e] = pack_bf16x2_pair(pp);
             }
-          };
-          chunk_p(std::integral_constant<bool, ACC>{});
+          }
           // The P region is free once the tile's previous PV products completed.
           if (pv_pending[t]) {
             if (!(ok = mbar_wait(&bar.pv_done[t], pvph[t], abort_flag, ws, 124))) break;
@@ -435,8 +428,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
     const uint32_t tS = tmem + lane_off + C::TM_S + t * 128 + h * 64;
     const uint32_t tO = tmem + lane_off + C::TM_O + t * D + h * (D / 2);
-    constexpr float half_scale = 0.5f * Scale<D>::value;
-    constexpr float neg_scale_l2e = -Scale<D>::value * 1.4426950408889634f;
+    const uint64_t scale_l2e2 = f2_splat(Scale<D>::value * kLog2e);
     uint32_t sph = 0, oph = 0, turn_ph = 0;
     bool ok = true;
     uint32_t ist = 0, iph = 0;
@@ -459,8 +451,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
         continue;
       }
       const int nkb = ceil_div(n, C::BN);
-      const float half_bias = -0.5f * __logf(static_cast<float>(n));
-      const float neg_bias_l2e = __log2f(static_cast<float>(n));  // -bias * log2(e)
+      const uint64_t neg_log2n2 = f2_splat(-__log2f(static_cast<float>(n)));  // bias * log2(e)
       for (int j = 0; j < nkb; ++j) {
         if (!(ok = mbar_wait(&bar.s_full[t], sph, abort_flag, ws, 121))) break;
         sph ^= 1;
@@ -480,21 +471,17 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           uint32_t a[32];
           tmem_ld32(tS + 32 * c, a);
           uint32_t pk[16];
-          auto chunk_p = [&](auto accurate) {
-            constexpr bool kAcc = decltype(accurate)::value;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float p0 = sigmoid_of<kAcc>(__uint_as_float(a[2 * e]), half_scale, half_bias, neg_scale_l2e, neg_bias_l2e);
-              float p1 =
-                  sigmoid_of<kAcc>(__uint_as_float(a[2 * e + 1]), half_scale, half_bias, neg_scale_l2e, neg_bias_l2e);
-              if (valid < 64) {
-                p0 = (32 * c + 2 * e < valid) ? p0 : 0.f;
-                p1 = (32 * c + 2 * e + 1 < valid) ? p1 : 0.f;
-              }
-              pk[e] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t pp = sigmoid2<false>(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]), scale_l2e2,
+                                                neg_log2n2, nullptr);
+            if (valid < 64) {
+              const float2 p = f2_unpack(pp);
+              pk[e] = pack_bf16x2((32 * c + 2 * e < valid) ? p.x : 0.f, (32 * c + 2 * e + 1 < valid) ? p.y : 0.f);
+            } else {
+              pk[e] = pack_bf16x2_pair(pp);
             }
-          };
-          chunk_p(std::integral_constant<bool, ACC>{});
+          }
           tmem_st16(tS + 16 * c, pk);
         }
         tmem_st_wait();
@@ -538,42 +525,31 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
   }
 }
 
-template <int D, bool PACKED, bool ACC>
+template <int D, bool PACKED>
 cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
                             int B, int H, int L, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D>;
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, PACKED, ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static PerDeviceOnce attr;
+  const cudaError_t e = attr.run([] {
+    return cudaFuncSetAttribute(fwd_kernel<D, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_ALLOC);
+  });
+  if (e != cudaSuccess) return e;
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kFwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
-  return launch_programmatic(fwd_kernel<D, PACKED, ACC>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, tq, tk,
+  return launch_programmatic(fwd_kernel<D, PACKED>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, tq, tk,
                              tv, static_cast<__nv_bfloat16*>(o), ws, H, L);
-}
-
-template <int D, bool PACKED>
-cudaError_t launch_fwd_layout(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
-                              int B, int H, int L, int num_sms, cudaStream_t stream) {
-  // No sequence is longer than L, so L decides the sigmoid route for the call.
-  if (L > kAccurateSigmoidLen) return launch_fwd_impl<D, PACKED, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
-  return launch_fwd_impl<D, PACKED, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
 }
 
 // L is Lmax for the padded layout and the longest sequence for the packed one.
 cudaError_t launch_fwd(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        void* o, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream) {
   if (packed) {
-    if (d == 64) return launch_fwd_layout<64, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
-    return launch_fwd_layout<128, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+    if (d == 64) return launch_fwd_impl<64, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+    return launch_fwd_impl<128, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
   }
-  if (d == 64) return launch_fwd_layout<64, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
-  return launch_fwd_layout<128, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+  if (d == 64) return launch_fwd_impl<64, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+  return launch_fwd_impl<128, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
 }
 
 }  // namespace sigattn

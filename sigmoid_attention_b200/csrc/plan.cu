@@ -118,15 +118,12 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
 cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, int* ws,
                         cudaStream_t stream) {
   const int smem = (4 * B + 1) * static_cast<int>(sizeof(int));
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (4 * kMaxBatch + 1) * static_cast<int>(sizeof(int)));
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static PerDeviceOnce attr;
+  const cudaError_t e = attr.run([] {
+    return cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (4 * kMaxBatch + 1) * static_cast<int>(sizeof(int)));
+  });
+  if (e != cudaSuccess) return e;
   const int threads = B <= 256 ? 256 : 1024;
   prep_kernel<<<1, threads, smem, stream>>>(lengths, cu, total, B, H, L, item_rows(kind), ws);
   return cudaGetLastError();
@@ -174,6 +171,32 @@ __global__ void selftest_timeout_kernel(int* ws, unsigned long long limit_ns) {
 
 cudaError_t launch_selftest_timeout(int* ws, unsigned long long limit_ns, cudaStream_t stream) {
   selftest_timeout_kernel<<<1, 32, 0, stream>>>(ws, limit_ns);
+  return cudaGetLastError();
+}
+
+// Diagnostic: the sigmoid of scores exactly as the compute kernels evaluate it
+// (sigmoid_score with the kernels' constants for head size D and length n),
+// and its derivative as the backward kernels use it.
+template <int D>
+__global__ void eval_sigmoid_kernel(const float* __restrict__ s, float* __restrict__ p, float* __restrict__ slope,
+                                    int count, int n) {
+  const float scale_l2e = Scale<D>::value * kLog2e;
+  const float neg_log2n = -__log2f(static_cast<float>(n));
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x) {
+    float dp;
+    const float v = sigmoid_score(s[i], scale_l2e, neg_log2n, &dp);
+    p[i] = v;
+    slope[i] = dp;
+  }
+}
+
+cudaError_t launch_eval_sigmoid(const float* s, float* p, float* slope, int count, int d, int n, int num_sms,
+                                cudaStream_t stream) {
+  const int grid = std::max(1, std::min(4 * num_sms, ceil_div(count, 256)));
+  if (d == 64)
+    eval_sigmoid_kernel<64><<<grid, 256, 0, stream>>>(s, p, slope, count, n);
+  else
+    eval_sigmoid_kernel<128><<<grid, 256, 0, stream>>>(s, p, slope, count, n);
   return cudaGetLastError();
 }
 
