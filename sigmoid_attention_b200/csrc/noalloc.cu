@@ -22,6 +22,9 @@
 
 namespace sigattn {
 void set_last_error(const char* msg);
+int check_fwd_inputs(const void* q, const void* k, const void* v, const void* o, const int32_t* lengths, int B,
+                     int H, int L, int d);
+int report_cuda(cudaError_t e);
 }
 
 namespace {
@@ -31,7 +34,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[SIGATTN_NOALLOC
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
-
 
 // Device address of the scratch array on the current device (set up on the
 // first call per device). Returns nullptr on failure.
@@ -57,8 +59,12 @@ void* scratch_address(cudaError_t* err) {
 
 extern "C" int sigattn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, const int32_t* lengths,
                                    int B, int H, int Lmax, int d, int32_t* status_out, void* stream) {
+  // Every argument check comes first, so that a rejected call leaves the
+  // shared array and the stream untouched.
+  int st = sigattn::check_fwd_inputs(q, k, v, o, lengths, B, H, Lmax, d);
+  if (st != SIGATTN_OK) return st;
+  if (status_out != nullptr && (reinterpret_cast<uintptr_t>(status_out) & 3u) != 0) return SIGATTN_ERR_INVALID_ARG;
   const size_t need = sigattn_workspace_size(B, H, Lmax, d);
-  if (need == 0) return (d != 64 && d != 128) ? SIGATTN_ERR_UNSUPPORTED : SIGATTN_ERR_INVALID_ARG;
   if (need > static_cast<size_t>(SIGATTN_NOALLOC_SCRATCH_BYTES)) {
     // B * H * ceil(Lmax / 128) work items do not fit the fixed scratch array.
     char msg[160];
@@ -69,20 +75,13 @@ extern "C" int sigattn_fwd_noalloc(const void* q, const void* k, const void* v, 
   }
   cudaError_t err = cudaSuccess;
   void* scratch = scratch_address(&err);
-  if (scratch == nullptr) {
-    char msg[160];
-    snprintf(msg, sizeof(msg), "sigattn_fwd_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(err));
-    sigattn::set_last_error(msg);
-    return SIGATTN_ERR_CUDA;
-  }
+  if (scratch == nullptr) return sigattn::report_cuda(err);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // The array keeps whatever the previous call left; the status words must
   // start at zero for this call.
-  if (cudaMemsetAsync(scratch, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SIGATTN_ERR_CUDA;
-  const int st = sigattn_fwd(q, k, v, o, lengths, B, H, Lmax, d, scratch, SIGATTN_NOALLOC_SCRATCH_BYTES, stream);
+  st = sigattn::report_cuda(cudaMemsetAsync(scratch, 0, 2 * sizeof(int32_t), s));
   if (st != SIGATTN_OK) return st;
-  if (status_out != nullptr &&
-      cudaMemcpyAsync(status_out, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-    return SIGATTN_ERR_CUDA;
-  return SIGATTN_OK;
+  st = sigattn_fwd(q, k, v, o, lengths, B, H, Lmax, d, scratch, SIGATTN_NOALLOC_SCRATCH_BYTES, stream);
+  if (st != SIGATTN_OK || status_out == nullptr) return st;
+  return sigattn::report_cuda(cudaMemcpyAsync(status_out, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
 }
