@@ -9,10 +9,11 @@ count) divided by the device time of the timed steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-With N > 1 (launched by torch.distributed.run, one process per GPU) every rank
-runs its own batch of the same workload: the (b, h) slices are independent, so
-the work shards with no collective on the data path (weak scaling). Rank 0
-prints one JSON line.
+With N > 1 every rank (one process per GPU, started by torch.distributed.run;
+bench.py starts that launcher itself when it was not started by one) runs its
+own batch of the same workload: the (b, h) slices are independent, so the work
+shards with no collective on the data path (weak scaling). Rank 0 prints one
+JSON line. A launcher whose WORLD_SIZE differs from --gpus is an error.
 """
 from __future__ import annotations
 
@@ -228,6 +229,146 @@ def run_reference(args, w):
     return 0
 
 
+def _run_calls(calls, stream, ev=None):
+    """One step: the forward, dQ and dK/dV calls, with an event before each
+    call and after the last when `ev` (four CUDA events) is given."""
+    for i, call in enumerate(calls):
+        if ev is not None:
+            ev[i].record(stream)
+        call()
+    if ev is not None:
+        ev[len(calls)].record(stream)
+
+
+def _check_status(sa, ws, stream):
+    st, site = sa.sigattn_read_error(ws, stream)
+    if st != 0:
+        raise SystemExit(f"kernel reported status {st} at site {site}")
+
+
+def _device_steps(calls, stream, steps, warmup, flush_buf=None, sync_ranks=None, check=None, sampler=None):
+    """Device time of each call over `steps` timed steps after `warmup`
+    untimed ones: CUDA events on the launching stream, a synchronize (and a
+    barrier over ranks, when given) on both sides of the timed region, and an
+    L2 flush (a write of flush_buf) between steps outside the events. A clock
+    `sampler` (context manager) runs during the timed region only."""
+    import contextlib
+
+    import torch
+
+    for _ in range(warmup):
+        _run_calls(calls, stream)
+        if flush_buf is not None:
+            flush_buf.zero_()
+    if check is not None:
+        check()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    if sync_ranks is not None:
+        sync_ranks()
+    torch.cuda.synchronize()
+    with sampler if sampler is not None else contextlib.nullcontext():
+        for i in range(steps):
+            _run_calls(calls, stream, events[i])
+            if flush_buf is not None:
+                flush_buf.zero_()
+        torch.cuda.synchronize()
+    if sync_ranks is not None:
+        sync_ranks()
+    if check is not None:
+        check()
+    per_kernel = {"fwd": [], "bwd_dq": [], "bwd_dkdv": []}
+    step_ms = []
+    for ev in events:
+        per_kernel["fwd"].append(ev[0].elapsed_time(ev[1]))
+        per_kernel["bwd_dq"].append(ev[1].elapsed_time(ev[2]))
+        per_kernel["bwd_dkdv"].append(ev[2].elapsed_time(ev[3]))
+        step_ms.append(ev[0].elapsed_time(ev[3]))
+    return per_kernel, step_ms
+
+
+def side_workloads(names, dev, steps: int, warmup: int) -> dict:
+    """Device-timed fwd / bwd / step TFLOPS of other workloads in the same run
+    (padded layout, L2 flushed between steps), with the padding-sweep ratio
+    of 75 % padding to unpadded."""
+    import torch
+
+    import sigmoid_attention_b200 as sa
+    from sigmoid_attention_b200 import workloads
+
+    out = {}
+    stream = torch.cuda.current_stream(dev)
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    for name in names:
+        w = workloads.WORKLOADS[name]
+        q, k, v, dout, lengths = workloads.workload_inputs(w)
+        qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, dout))
+        lens = lengths.to(dev)
+        o, dq, dk, dv = (torch.empty_like(qd) for _ in range(4))
+        ws = sa.make_workspace(w.B, w.H, w.L, w.d, dev)
+        calls = (lambda: sa.sigattn_fwd(qd, kd, vd, o, lens, ws, stream),
+                 lambda: sa.sigattn_bwd_dq(qd, kd, vd, dod, dq, lens, ws, stream),
+                 lambda: sa.sigattn_bwd_dkdv(qd, kd, vd, dod, dk, dv, lens, ws, stream))
+        per_kernel, step_ms = _device_steps(calls, stream, steps, warmup, flush_buf,
+                                            check=lambda: _check_status(sa, ws, stream))
+        f_fwd, f_bwd = w.fwd_flops(), w.bwd_flops()
+        ms = {kname: float(np.mean(v_)) for kname, v_ in per_kernel.items()}
+        out[name] = {"value": (f_fwd + f_bwd) / (np.mean(step_ms) / 1e3) / 1e12,
+                     "fwd_tflops": f_fwd / (ms["fwd"] / 1e3) / 1e12,
+                     "bwd_tflops": f_bwd / ((ms["bwd_dq"] + ms["bwd_dkdv"]) / 1e3) / 1e12,
+                     "ms": ms, "steps": steps}
+        del qd, kd, vd, dod, o, dq, dk, dv, ws
+    if "pad_sweep_p00" in out and "pad_sweep_p75" in out:
+        out["p75_over_p00"] = out["pad_sweep_p75"]["value"] / out["pad_sweep_p00"]["value"]
+    return out
+
+
+def unfused_torch(w, q, k, v, dout, lengths, dev, steps: int = 5, warmup: int = 3) -> dict:
+    """The comparison of "Better Models, Faster Training" sec. 4A: sigmoid
+    attention written as plain PyTorch operations (bf16 matmuls, an explicit
+    score tensor, sigmoid, mask, matmul; backward by autograd) on the same
+    inputs, timed the same way, with the same valid-pair FLOP count. It is a
+    baseline for the speed-up figures, not part of the library."""
+    import math as _m
+
+    import torch
+
+    B, H, L, d = q.shape
+    qd, kd, vd, dod = (t.to(dev).requires_grad_(i < 3) for i, t in enumerate((q, k, v, dout)))
+    n = lengths.to(dev).to(torch.float32)
+    bias = (-torch.log(n.clamp_min(1))).view(B, 1, 1, 1).to(torch.bfloat16)
+    idx = torch.arange(L, device=dev)
+    valid = idx.view(1, L) < lengths.to(dev).view(B, 1)
+    mask = (valid.view(B, 1, L, 1) & valid.view(B, 1, 1, L))
+
+    def fwd():
+        s_ = torch.matmul(qd, kd.transpose(-1, -2)) * (1.0 / _m.sqrt(d)) + bias
+        p_ = torch.where(mask, torch.sigmoid(s_), torch.zeros((), dtype=s_.dtype, device=dev))
+        return torch.matmul(p_, vd)
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    fwd_ms, bwd_ms = [], []
+    for i in range(warmup + steps):
+        for t in (qd, kd, vd):
+            t.grad = None
+        ev[0].record()
+        out = fwd()
+        ev[1].record()
+        out.backward(dod)
+        ev[2].record()
+        torch.cuda.synchronize(dev)
+        if i >= warmup:
+            fwd_ms.append(ev[0].elapsed_time(ev[1]))
+            bwd_ms.append(ev[1].elapsed_time(ev[2]))
+    f_fwd, f_bwd = w.fwd_flops(), w.bwd_flops()
+    res = {"fwd_ms": float(np.mean(fwd_ms)), "bwd_ms": float(np.mean(bwd_ms)),
+           "fwd_tflops": f_fwd / (np.mean(fwd_ms) / 1e3) / 1e12, "bwd_tflops": f_bwd / (np.mean(bwd_ms) / 1e3) / 1e12,
+           "steps": steps, "what": "torch.matmul (bf16) -> scale + bias -> sigmoid -> mask -> torch.matmul; "
+                                   "backward by autograd"}
+    del qd, kd, vd, dod, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def pcie_bandwidth(dev, nbytes: int = 256 << 20, reps: int = 6) -> dict:
     """Pinned host <-> device copy bandwidth in GB/s: each direction alone, and
     per direction with both running at once (the bound of a pipelined step)."""
@@ -299,58 +440,22 @@ def run_gpu(args, w):
     flush = footprint < 4 * L2_BYTES
     scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
 
+    if packed:
+        calls = (lambda: sa.sigattn_fwd_varlen(qd, kd, vd, o, lens, max_seqlen, ws, stream),
+                 lambda: sa.sigattn_bwd_dq_varlen(qd, kd, vd, dod, dq, lens, max_seqlen, ws, stream),
+                 lambda: sa.sigattn_bwd_dkdv_varlen(qd, kd, vd, dod, dk, dv, lens, max_seqlen, ws, stream))
+    else:
+        calls = (lambda: sa.sigattn_fwd(qd, kd, vd, o, lens, ws, stream),
+                 lambda: sa.sigattn_bwd_dq(qd, kd, vd, dod, dq, lens, ws, stream),
+                 lambda: sa.sigattn_bwd_dkdv(qd, kd, vd, dod, dk, dv, lens, ws, stream))
+
     def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        if packed:
-            sa.sigattn_fwd_varlen(qd, kd, vd, o, lens, max_seqlen, ws, stream)
-        else:
-            sa.sigattn_fwd(qd, kd, vd, o, lens, ws, stream)
-        if ev is not None:
-            ev[1].record(stream)
-        if packed:
-            sa.sigattn_bwd_dq_varlen(qd, kd, vd, dod, dq, lens, max_seqlen, ws, stream)
-        else:
-            sa.sigattn_bwd_dq(qd, kd, vd, dod, dq, lens, ws, stream)
-        if ev is not None:
-            ev[2].record(stream)
-        if packed:
-            sa.sigattn_bwd_dkdv_varlen(qd, kd, vd, dod, dk, dv, lens, max_seqlen, ws, stream)
-        else:
-            sa.sigattn_bwd_dkdv(qd, kd, vd, dod, dk, dv, lens, ws, stream)
-        if ev is not None:
-            ev[3].record(stream)
+        _run_calls(calls, stream, ev)
 
-    for _ in range(args.warmup):
-        step()
-        if flush:
-            scratch.zero_()
-    st, site = sa.sigattn_read_error(ws, stream)
-    if st != 0:
-        raise SystemExit(f"kernel reported status {st} at site {site}")
-
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
-        for i in range(args.steps):
-            step(events[i])
-            if flush:
-                scratch.zero_()
-        torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    per_kernel = {"fwd": [], "bwd_dq": [], "bwd_dkdv": []}
-    step_ms = []
-    for ev in events:
-        per_kernel["fwd"].append(ev[0].elapsed_time(ev[1]))
-        per_kernel["bwd_dq"].append(ev[1].elapsed_time(ev[2]))
-        per_kernel["bwd_dkdv"].append(ev[2].elapsed_time(ev[3]))
-        step_ms.append(ev[0].elapsed_time(ev[3]))
-    st, site = sa.sigattn_read_error(ws, stream)
-    if st != 0:
-        raise SystemExit(f"kernel reported status {st} at site {site}")
+    sync_ranks = (lambda: torch.distributed.barrier()) if world > 1 else None
+    clocks = ClockSampler(local)
+    per_kernel, step_ms = _device_steps(calls, stream, args.steps, args.warmup, scratch, sync_ranks,
+                                        lambda: _check_status(sa, ws, stream), clocks)
     total_s = reduce_max(sum(step_ms) / 1e3, world, dev)
     fwd_s = reduce_max(sum(per_kernel["fwd"]) / 1e3, world, dev)
     bwd_s = reduce_max((sum(per_kernel["bwd_dq"]) + sum(per_kernel["bwd_dkdv"])) / 1e3, world, dev)
@@ -502,6 +607,20 @@ def run_gpu(args, w):
         "gpu_launches": (6 if packed else 8) * args.steps,
         "clocks": clk,
     }
+    if world == 1 and not args.no_extras:
+        # Same run, same box: the padding ratio and the short-sequence workloads
+        # (device-timed), and the unfused PyTorch comparison on this workload.
+        side = [n_ for n_ in ("pad_sweep_p00", "pad_sweep_p75", "scrna_ragged", "long_8k") if n_ != w.name]
+        line["other_workloads"] = side_workloads(side, dev, steps=10, warmup=3)
+        if w.name in ("pad_sweep_p00", "pad_sweep_p75"):
+            mine = {"value": value, "fwd_tflops": fwd_tflops, "bwd_tflops": bwd_tflops}
+            other = line["other_workloads"].get("pad_sweep_p75" if w.name == "pad_sweep_p00" else "pad_sweep_p00")
+            p00, p75 = (mine, other) if w.name == "pad_sweep_p00" else (other, mine)
+            line["other_workloads"]["p75_over_p00"] = p75["value"] / p00["value"]
+        if not packed:
+            u = unfused_torch(w, q, k, v, dout, lengths, dev)
+            u["fused_speedup"] = {"fwd": fwd_tflops / u["fwd_tflops"], "bwd": bwd_tflops / u["bwd_tflops"]}
+            line["unfused_torch"] = u
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -510,6 +629,34 @@ def run_gpu(args, w):
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     return 0
+
+
+def spawn_ranks(n: int, argv: list, timeout_s: float = 3600.0) -> int:
+    """Run this script as n ranks (one process per GPU) under
+    torch.distributed.run on this node, rendezvous on 127.0.0.1, and return
+    the launcher's exit code. The launcher and its ranks form one process
+    group, which is ended as a whole if it outlives `timeout_s`."""
+    import signal
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "LOCAL_RANK", "WORLD_SIZE")}
+    proc = subprocess.Popen(cmd, env=env, start_new_session=True)
+    try:
+        return proc.wait(timeout=timeout_s)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGTERM)
+        try:
+            proc.wait(timeout=60)
+        except subprocess.TimeoutExpired:
+            os.killpg(proc.pid, signal.SIGKILL)
+            proc.wait()
+        print(f"bench.py: {n}-rank run exceeded {timeout_s:.0f} s", file=sys.stderr)
+        return 1
 
 
 def main(argv=None):
@@ -524,13 +671,20 @@ def main(argv=None):
     ap.add_argument("--layout", default="padded", choices=["padded", "packed"],
                     help="padded [B,H,Lmax,d] tensors, or the workload's valid tokens packed as [total,H,d]")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads and the unfused PyTorch comparison (1-GPU runs only)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = workloads.WORKLOADS[args.workload]
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # Not started by a launcher: start one process per GPU ourselves.
+        return spawn_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv))
     world, _, _ = _dist_env()
     if world != args.gpus:
-        print(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but the launcher started WORLD_SIZE={world} ranks")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

@@ -60,3 +60,37 @@ def test_single_rank_identity():
 
     assert bench.reduce_max(3.5, 1) == 3.5
     assert bench.whole_job_tflops(2e12, 1, 2.0) == pytest.approx(1.0)
+
+
+def _bench_env():
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR",
+                                                            "MASTER_PORT")}
+    env["CUDA_VISIBLE_DEVICES"] = ""
+    return env
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` without a launcher starts two ranks itself; the
+    line rank 0 prints counts both (the reference arm needs no GPU)."""
+    import json
+    import subprocess
+
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                          "--workload", "tiny", "--steps", "3", "--warmup", "3"], cwd=ROOT, env=_bench_env(),
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_gpus_flag_must_match_the_launcher():
+    import subprocess
+
+    env = _bench_env()
+    env.update(WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                          "--workload", "tiny", "--steps", "3", "--warmup", "3"], cwd=ROOT, env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode != 0
+    assert "WORLD_SIZE=1" in out.stderr
