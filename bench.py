@@ -582,7 +582,7 @@ def run_gpu(args, w):
                    "step": ("sigattn_fwd_varlen + sigattn_bwd_dq_varlen + sigattn_bwd_dkdv_varlen "
                             "(each: plan + compute kernel)") if packed else
                            ("sigattn_fwd + sigattn_bwd_dq + sigattn_bwd_dkdv "
-                            "(each: plan + compute kernel; zero-fill kernel after fwd and dK/dV)"),
+                            "(each: plan + compute kernel; zero-fill kernel beside the forward)"),
                    "flops": "valid pairs only: 4*d fwd + 10*d bwd per pair",
                    "parallelism": f"replica per GPU x{world} (independent batches)",
                    "l2": ("flushed between steps (footprint %.0f MB)" % (footprint / 1e6)) if flush else
@@ -603,8 +603,8 @@ def run_gpu(args, w):
         "e2e_serial": {"value": e2e_serial, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "steps": e2e_steps, "schedule": "copy in, three calls, copy out, one stream"},
         # Device-timed steps only: per call the plan and compute kernels, plus (padded
-        # layout) the zero-fill kernel after the forward and dK/dV kernels.
-        "gpu_launches": (6 if packed else 8) * args.steps,
+        # layout) the zero-fill kernel beside the forward kernel.
+        "gpu_launches": (6 if packed else 7) * args.steps,
         "clocks": clk,
     }
     if world == 1 and not args.no_extras:

@@ -112,6 +112,47 @@ SIGATTN_API int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, co
                      const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* Key ranges: the padded-layout calls restricted to the keys at positions
+ * [key_begin, key_begin + key_count) of every sequence, for attention whose
+ * keys are split over several calls or GPUs (sequence sharding). Because each
+ * weight sigma(q.k/sqrt(d) - ln n) stands on its own, with no normalisation
+ * over the keys (sec. 2A), O = sigma(S + b) V is the plain sum over key ranges
+ * of each range's contribution, and so is dQ = scale dS K (sec. 2B/2C); dK and
+ * dV of a key depend on that key and on all queries only. The bias still uses
+ * each sequence's full length n_b.
+ *  - q, dout: [B][H][Lmax][d] bf16, all query rows. k, v: [B][H][key_count][d]
+ *    bf16 holding keys key_begin .. key_begin + key_count - 1 of every
+ *    sequence; a key at position key_begin + j is valid if it is < n_b.
+ *  - 0 <= key_begin, 1 <= key_count, key_begin + key_count <= Lmax; the
+ *    workspace is sigattn_workspace_size(B, H, Lmax, d) as usual.
+ *  - sigattn_fwd_partial writes o_partial [B][H][Lmax][d] fp32 (16-byte
+ *    aligned): for valid rows i the sum over the range's valid keys j of
+ *    P_ij V_j, not rounded; rows i >= n_b, and every row of a sequence with no
+ *    valid key in the range, are 0. Summing the partials of ranges that tile
+ *    [0, Lmax) gives O in fp32.
+ *  - sigattn_bwd_dq_partial writes dq_partial [B][H][Lmax][d] fp32 likewise:
+ *    the range's share of dQ, scale included.
+ *  - sigattn_bwd_dkdv_range writes dk, dv [B][H][key_count][d] bf16: the rows
+ *    of dK and dV for the range's keys (zero for keys >= n_b). With
+ *    key_begin a multiple of 128 they are the same bits as the matching rows
+ *    of sigattn_bwd_dkdv.
+ *  - Everything else as for sigattn_fwd / sigattn_bwd_dq / sigattn_bwd_dkdv. */
+SIGATTN_API int sigattn_fwd_partial(const void* q, const void* k, const void* v, float* o_partial,
+                                    const int32_t* lengths, int B, int H, int Lmax, int d, int key_begin,
+                                    int key_count, void* workspace, size_t workspace_bytes, void* stream);
+SIGATTN_API int sigattn_bwd_dq_partial(const void* q, const void* k, const void* v, const void* dout,
+                                       float* dq_partial, const int32_t* lengths, int B, int H, int Lmax, int d,
+                                       int key_begin, int key_count, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+SIGATTN_API int sigattn_bwd_dkdv_range(const void* q, const void* k, const void* v, const void* dout, void* dk,
+                                       void* dv, const int32_t* lengths, int B, int H, int Lmax, int d, int key_begin,
+                                       int key_count, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Round `count` fp32 values to bf16 (nearest even), x -> y, both device
+ * pointers, 16-byte aligned; count a multiple of 8. The last step after the
+ * fp32 partial sums of key ranges were added (e.g. by an all-reduce). */
+SIGATTN_API int sigattn_cast_bf16(const float* x, void* y, long long count, void* stream);
+
 /* Packed ("varlen") layout: the same three operations on sequences stored
  * back to back instead of padded to Lmax, so padding costs neither FLOPs nor
  * HBM bytes. Sequence b's tokens are rows cu_seqlens[b] .. cu_seqlens[b+1]-1

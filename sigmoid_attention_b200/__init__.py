@@ -23,6 +23,7 @@ __all__ = [
     "sigattn_workspace_size", "sigattn_fwd", "sigattn_fwd_noalloc", "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
     "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "sigattn_eval_sigmoid", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
     "sigattn_fwd_varlen", "sigattn_bwd_dq_varlen", "sigattn_bwd_dkdv_varlen",
+    "sigattn_fwd_partial", "sigattn_bwd_dq_partial", "sigattn_bwd_dkdv_range", "sigattn_cast_bf16",
     "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
     "SigmoidAttentionVarlenFunction", "sigmoid_attention_varlen",
 ]
@@ -87,6 +88,14 @@ def library():
         lib.sigattn_selftest_wait_timeout.argtypes = [_vp, _sz, _i, _vp]
         lib.sigattn_last_error.restype = ctypes.c_char_p
         lib.sigattn_last_error.argtypes = []
+        lib.sigattn_fwd_partial.restype = _i
+        lib.sigattn_fwd_partial.argtypes = [_vp] * 5 + [_i] * 6 + [_vp, _sz, _vp]
+        lib.sigattn_bwd_dq_partial.restype = _i
+        lib.sigattn_bwd_dq_partial.argtypes = [_vp] * 6 + [_i] * 6 + [_vp, _sz, _vp]
+        lib.sigattn_bwd_dkdv_range.restype = _i
+        lib.sigattn_bwd_dkdv_range.argtypes = [_vp] * 7 + [_i] * 6 + [_vp, _sz, _vp]
+        lib.sigattn_cast_bf16.restype = _i
+        lib.sigattn_cast_bf16.argtypes = [_vp, _vp, ctypes.c_longlong, _vp]
         lib.sigattn_eval_sigmoid.restype = _i
         lib.sigattn_eval_sigmoid.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp]
         lib.sigattn_read_error.restype = _i
@@ -176,6 +185,41 @@ def sigattn_bwd_dkdv(q, k, v, dout, dk, dv, lengths, workspace, stream=None) -> 
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dk, "dk"), _dev(dv, "dv"),
         _dev(lengths, "lengths", torch.int32), B, H, L, d, _dev(workspace, "workspace", torch.uint8),
         workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_fwd_partial(q, k, v, o_partial, lengths, key_begin: int, workspace, stream=None) -> None:
+    """Key-range forward: k, v are [B, H, key_count, d] bf16 holding keys
+    key_begin .. key_begin + key_count - 1 of every sequence; o_partial is the
+    fp32 [B, H, Lmax, d] contribution of those keys (see the C header)."""
+    B, H, L, d = _dims(q)
+    _check("sigattn_fwd_partial", library().sigattn_fwd_partial(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o_partial, "o_partial", torch.float32),
+        _dev(lengths, "lengths", torch.int32), B, H, L, d, int(key_begin), int(k.shape[2]),
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_bwd_dq_partial(q, k, v, dout, dq_partial, lengths, key_begin: int, workspace, stream=None) -> None:
+    B, H, L, d = _dims(q)
+    _check("sigattn_bwd_dq_partial", library().sigattn_bwd_dq_partial(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dq_partial, "dq_partial", torch.float32),
+        _dev(lengths, "lengths", torch.int32), B, H, L, d, int(key_begin), int(k.shape[2]),
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_bwd_dkdv_range(q, k, v, dout, dk, dv, lengths, key_begin: int, workspace, stream=None) -> None:
+    B, H, L, d = _dims(q)
+    _check("sigattn_bwd_dkdv_range", library().sigattn_bwd_dkdv_range(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dk, "dk"), _dev(dv, "dv"),
+        _dev(lengths, "lengths", torch.int32), B, H, L, d, int(key_begin), int(k.shape[2]),
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_cast_bf16(x, y, stream=None) -> None:
+    """y (bf16) = x (fp32) rounded to nearest even; same number of elements."""
+    if x.numel() != y.numel():
+        raise ValueError("x and y must have the same number of elements")
+    _check("sigattn_cast_bf16", library().sigattn_cast_bf16(
+        _dev(x, "x", torch.float32), _dev(y, "y"), x.numel(), _stream_ptr(stream)))
 
 
 def _packed_dims(q: torch.Tensor):

@@ -12,22 +12,24 @@
 #include "common.cuh"
 
 namespace sigattn {
-cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, int* ws,
-                        cudaStream_t stream);
-cudaError_t launch_fill(const int* lengths, int B, int H, int L, int d, int kind, void* out0, void* out1,
-                        int num_sms, cudaStream_t stream);
+cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, KeyRange kr,
+                        int* ws, cudaStream_t stream);
+cudaError_t launch_fill(const int* lengths, int B, int H, int L, int d, int kind, KeyRange kr, int elem_bytes,
+                        void* out0, void* out1, int num_sms, cudaStream_t stream);
 int plan_host(const int* lengths, int B, int H, int L, int kind, int* out, int cap);
 cudaError_t launch_selftest_timeout(int* ws, unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_eval_sigmoid(const float* s, float* p, float* slope, int count, int d, int n, int num_sms,
                                 cudaStream_t stream);
-cudaError_t launch_fwd(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       void* o, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream);
-cudaError_t launch_bwd_dq(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                          const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L, int num_sms,
-                          const int* fill_lengths, cudaStream_t stream);
+cudaError_t launch_cast_bf16(const float* in, void* out, long long count, int num_sms, cudaStream_t stream);
+cudaError_t launch_fwd(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, void* o, int* ws, int B, int H, int L, KeyRange kr, int num_sms,
+                       cudaStream_t stream);
+cudaError_t launch_bwd_dq(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tdo,
+                          const CUtensorMap& tk, const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L,
+                          KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream);
 cudaError_t launch_bwd_dkdv(int d, bool packed, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                            const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int L, int num_sms,
-                            cudaStream_t stream);
+                            const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int out_rows, int Lmax,
+                            KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream);
 void set_last_error(const char* msg);
 }  // namespace sigattn
 
@@ -171,6 +173,83 @@ int check_call(int B, int H, int L, int d, const int32_t* lengths, const void* w
   return SIGATTN_OK;
 }
 
+// The key range of a padded-layout call: 0 <= begin, 1 <= count and
+// begin + count <= Lmax.
+bool range_ok(KeyRange kr, int Lmax) {
+  return kr.begin >= 0 && kr.count >= 1 && static_cast<long long>(kr.begin) + kr.count <= Lmax;
+}
+
+// Padded-layout forward over the keys kr (whole sequences: {0, Lmax}); k and
+// v hold those keys only ([B][H][kr.count][d]); f32out writes o as fp32.
+int fwd_padded(const void* q, const void* k, const void* v, void* o, bool f32out, const int32_t* lengths, int B,
+               int H, int Lmax, int d, KeyRange kr, void* workspace, size_t workspace_bytes, void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (!range_ok(kr, Lmax)) return SIGATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SIGATTN_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, kr.count, d) ||
+      !make_map(&tv, v, B * H, kr.count, d))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_FWD, kr, ws, s));
+  if (st == SIGATTN_OK)
+    st = cuda_status(launch_fwd(d, false, f32out, tq, tk, tv, o, ws, B, H, Lmax, kr, info.num_sms, s));
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(
+      launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_FWD, kr, f32out ? 4 : 2, o, nullptr, info.num_sms, s));
+}
+
+int dq_padded(const void* q, const void* k, const void* v, const void* dout, void* dq, bool f32out,
+              const int32_t* lengths, int B, int H, int Lmax, int d, KeyRange kr, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (!range_ok(kr, Lmax)) return SIGATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq))
+    return SIGATTN_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, kr.count, d) ||
+      !make_map(&tv, v, B * H, kr.count, d) || !make_map(&tdo, dout, B * H, Lmax, d))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_DQ, kr, ws, s));
+  if (st != SIGATTN_OK) return st;
+  // The dQ kernel zeroes dQ's uncovered padded rows itself.
+  return cuda_status(
+      launch_bwd_dq(d, false, f32out, tq, tdo, tk, tv, dq, ws, B, H, Lmax, kr, info.num_sms, lengths, s));
+}
+
+// dK, dV of the keys kr: k, v, dk, dv are [B][H][kr.count][d].
+int dkdv_padded(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                const int32_t* lengths, int B, int H, int Lmax, int d, KeyRange kr, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (!range_ok(kr, Lmax)) return SIGATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
+    return SIGATTN_ERR_INVALID_ARG;
+  // K, V are the row operands (128-row boxes); Q, dO are streamed in blocks of
+  // bwd_col_block(true, d) rows.
+  const int cb = bwd_col_block(true, d);
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, B * H, Lmax, d, cb) || !make_map(&tk, k, B * H, kr.count, d) ||
+      !make_map(&tv, v, B * H, kr.count, d) || !make_map(&tdo, dout, B * H, Lmax, d, cb))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_DKDV, kr, ws, s));
+  if (st != SIGATTN_OK) return st;
+  // The dK/dV kernel zeroes the uncovered rows of dK and dV itself.
+  return cuda_status(
+      launch_bwd_dkdv(d, false, tk, tv, tq, tdo, dk, dv, ws, B, H, kr.count, Lmax, kr, info.num_sms, lengths, s));
+}
+
 }  // namespace
 
 namespace sigattn {
@@ -225,62 +304,51 @@ size_t sigattn_workspace_size(int B, int H, int Lmax, int d) {
 
 int sigattn_fwd(const void* q, const void* k, const void* v, void* o, const int32_t* lengths, int B, int H,
                 int Lmax, int d, void* workspace, size_t workspace_bytes, void* stream) {
-  DeviceInfo info;
-  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
-  if (st != SIGATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SIGATTN_ERR_INVALID_ARG;
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) || !make_map(&tv, v, B * H, Lmax, d))
-    return map_failure();
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_FWD, ws, s));
-  if (st == SIGATTN_OK) st = cuda_status(launch_fwd(d, false, tq, tk, tv, o, ws, B, H, Lmax, info.num_sms, s));
-  if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_FWD, o, nullptr, info.num_sms, s));
+  return fwd_padded(q, k, v, o, false, lengths, B, H, Lmax, d, KeyRange{0, Lmax}, workspace, workspace_bytes, stream);
+}
+
+int sigattn_fwd_partial(const void* q, const void* k, const void* v, float* o_partial, const int32_t* lengths, int B,
+                        int H, int Lmax, int d, int key_begin, int key_count, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return fwd_padded(q, k, v, o_partial, true, lengths, B, H, Lmax, d, KeyRange{key_begin, key_count}, workspace,
+                    workspace_bytes, stream);
 }
 
 int sigattn_bwd_dq(const void* q, const void* k, const void* v, const void* dout, void* dq, const int32_t* lengths,
                    int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes, void* stream) {
-  DeviceInfo info;
-  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
-  if (st != SIGATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq))
-    return SIGATTN_ERR_INVALID_ARG;
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) ||
-      !make_map(&tv, v, B * H, Lmax, d) || !make_map(&tdo, dout, B * H, Lmax, d))
-    return map_failure();
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_DQ, ws, s));
-  if (st != SIGATTN_OK) return st;
-  // The dQ kernel zeroes dQ's uncovered padded rows itself.
-  return cuda_status(launch_bwd_dq(d, false, tq, tdo, tk, tv, dq, ws, B, H, Lmax, info.num_sms, lengths, s));
+  return dq_padded(q, k, v, dout, dq, false, lengths, B, H, Lmax, d, KeyRange{0, Lmax}, workspace, workspace_bytes,
+                   stream);
+}
+
+int sigattn_bwd_dq_partial(const void* q, const void* k, const void* v, const void* dout, float* dq_partial,
+                           const int32_t* lengths, int B, int H, int Lmax, int d, int key_begin, int key_count,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  return dq_padded(q, k, v, dout, dq_partial, true, lengths, B, H, Lmax, d, KeyRange{key_begin, key_count}, workspace,
+                   workspace_bytes, stream);
 }
 
 int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
                      const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes,
                      void* stream) {
+  return dkdv_padded(q, k, v, dout, dk, dv, lengths, B, H, Lmax, d, KeyRange{0, Lmax}, workspace, workspace_bytes,
+                     stream);
+}
+
+int sigattn_bwd_dkdv_range(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                           const int32_t* lengths, int B, int H, int Lmax, int d, int key_begin, int key_count,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  return dkdv_padded(q, k, v, dout, dk, dv, lengths, B, H, Lmax, d, KeyRange{key_begin, key_count}, workspace,
+                     workspace_bytes, stream);
+}
+
+int sigattn_cast_bf16(const float* x, void* y, long long count, void* stream) {
+  if (count < 0 || count % 8 != 0) return SIGATTN_ERR_INVALID_ARG;
+  if (count == 0) return SIGATTN_OK;
+  if (!aligned16(x) || !aligned16(y)) return SIGATTN_ERR_INVALID_ARG;
   DeviceInfo info;
-  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
-  if (st != SIGATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
-    return SIGATTN_ERR_INVALID_ARG;
-  // K, V are the row operands (128-row boxes); Q, dO are streamed in blocks of
-  // bwd_col_block(true, d) rows.
-  const int cb = bwd_col_block(true, d);
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, B * H, Lmax, d, cb) || !make_map(&tk, k, B * H, Lmax, d) ||
-      !make_map(&tv, v, B * H, Lmax, d) || !make_map(&tdo, dout, B * H, Lmax, d, cb))
-    return map_failure();
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_DKDV, ws, s));
-  if (st == SIGATTN_OK)
-    st = cuda_status(launch_bwd_dkdv(d, false, tk, tv, tq, tdo, dk, dv, ws, B, H, Lmax, info.num_sms, s));
-  if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_DKDV, dk, dv, info.num_sms, s));
+  if (!device_info(&info)) return cuda_status(cudaErrorUnknown);
+  if (!info.supported) return SIGATTN_ERR_UNSUPPORTED;
+  return cuda_status(launch_cast_bf16(x, y, count, info.num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 int sigattn_fwd_varlen(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens, int B,
@@ -297,9 +365,10 @@ int sigattn_fwd_varlen(const void* q, const void* k, const void* v, void* o, con
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_FWD, ws, s));
+  const KeyRange all{0, max_seqlen};
+  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_FWD, all, ws, s));
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_fwd(d, true, tq, tk, tv, o, ws, B, H, max_seqlen, info.num_sms, s));
+  return cuda_status(launch_fwd(d, true, false, tq, tk, tv, o, ws, B, H, max_seqlen, all, info.num_sms, s));
 }
 
 int sigattn_bwd_dq_varlen(const void* q, const void* k, const void* v, const void* dout, void* dq,
@@ -317,9 +386,11 @@ int sigattn_bwd_dq_varlen(const void* q, const void* k, const void* v, const voi
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_DQ, ws, s));
+  const KeyRange all{0, max_seqlen};
+  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_DQ, all, ws, s));
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_bwd_dq(d, true, tq, tdo, tk, tv, dq, ws, B, H, max_seqlen, info.num_sms, nullptr, s));
+  return cuda_status(
+      launch_bwd_dq(d, true, false, tq, tdo, tk, tv, dq, ws, B, H, max_seqlen, all, info.num_sms, nullptr, s));
 }
 
 int sigattn_bwd_dkdv_varlen(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
@@ -338,9 +409,11 @@ int sigattn_bwd_dkdv_varlen(const void* q, const void* k, const void* v, const v
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws = static_cast<int*>(workspace);
-  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_DKDV, ws, s));
+  const KeyRange all{0, max_seqlen};
+  st = cuda_status(launch_prep(nullptr, cu_seqlens, total, B, H, max_seqlen, SIGATTN_KIND_DKDV, all, ws, s));
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_bwd_dkdv(d, true, tk, tv, tq, tdo, dk, dv, ws, B, H, max_seqlen, info.num_sms, s));
+  return cuda_status(launch_bwd_dkdv(d, true, tk, tv, tq, tdo, dk, dv, ws, B, H, max_seqlen, max_seqlen, all,
+                                     info.num_sms, nullptr, s));
 }
 
 int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind, void* workspace,
@@ -349,7 +422,7 @@ int sigattn_plan(const int32_t* lengths, int B, int H, int Lmax, int d, int kind
   DeviceInfo info;
   int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
   if (st != SIGATTN_OK) return st;
-  return cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, kind, static_cast<int*>(workspace),
+  return cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, kind, KeyRange{0, Lmax}, static_cast<int*>(workspace),
                                  static_cast<cudaStream_t>(stream)));
 }
 

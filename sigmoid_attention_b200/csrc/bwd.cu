@@ -82,7 +82,16 @@ struct BwdCfg {
   static_assert(SMEM_ALLOC <= 227 * 1024 - 1024, "shared memory budget");
   static constexpr int EPI_WARPS = 8;
   static constexpr int ISSUERS = KV ? 4 : 3;
-  static constexpr int THREADS = (EPI_WARPS + 1 + ISSUERS) * 32;
+  // Four warpgroups: two of epilogue warps, then the producer, the issuers and
+  // idle warps. The single-thread roles give registers to the epilogue
+  // (setmaxnreg): launched at 128 per thread, 8 warps x 184 + 8 x 64 fit the
+  // 65536 registers of the SM.
+  static constexpr int THREADS = 16 * 32;
+  static constexpr int EPI_REGS = 184;
+  static constexpr int OTHER_REGS = 64;
+  static_assert(EPI_WARPS + 1 + ISSUERS <= 16, "warp roles");
+  static_assert((EPI_WARPS * EPI_REGS + (16 - EPI_WARPS) * OTHER_REGS) * 32 <= 65536, "register split");
+  static_assert(THREADS * 128 <= 65536, "launch registers");
 };
 
 template <int ST1, int ST2>
@@ -101,12 +110,16 @@ struct BwdBarriers {
   int abort;
 };
 
-template <int D, bool KV, bool PACKED>
+// kr: the keys the call covers (whole sequences: {0, Lmax}). For dQ the
+// columns are the range's keys; for dK/dV the rows are, and L is then the
+// rows per (b, h) slice of the dK/dV outputs (kr.count). F32OUT (dQ only):
+// write dQ as the fp32 partial sum over the range's keys.
+template <int D, bool KV, bool PACKED, bool F32OUT>
 __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_r1, const __grid_constant__ CUtensorMap tm_r2,
                const __grid_constant__ CUtensorMap tm_c1, const __grid_constant__ CUtensorMap tm_c2,
-               __nv_bfloat16* __restrict__ out1, __nv_bfloat16* __restrict__ out2,
-               int* __restrict__ ws, int H, int L, const int* __restrict__ fill_lengths, int B, int fill_parts) {
+               void* __restrict__ out1, void* __restrict__ out2, int* __restrict__ ws, int H, int L, KeyRange kr,
+               const int* __restrict__ fill_lengths, int B, int len_bound, int fill_parts) {
   using C = BwdCfg<D, KV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ BwdBarriers<C::ST1, C::ST2> bar;
@@ -160,6 +173,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   // 16-byte aligned addresses; the host already rejects outputs that are not,
   // and the check here keeps the rule next to the copies.
   const bool bulk_fill = C::ZBUF > 0 && fill_lengths != nullptr && (reinterpret_cast<uintptr_t>(out1) & 15u) == 0;
+  // Geometry of the zero fill of the output rows no item covers (dQ, or dK
+  // and dV); len_bound (Lmax) bounds the valid lengths.
+  const FillGeom fill_geom{H, len_bound, L, D * (F32OUT ? 4 : 2) / 16, KV ? kKindDkdv : kKindDq, C::BM, kr};
   if (bulk_fill) {
     uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_Z);
     for (int i = threadIdx.x; i < C::ZBUF / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
@@ -179,202 +195,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   const uint32_t sbase = smem_u32(smem);
   constexpr uint64_t kTileC = C::TILE_C >> 4;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------- producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_r1);
-      tma_prefetch_desc(&tm_r2);
-      tma_prefetch_desc(&tm_c1);
-      tma_prefetch_desc(&tm_c2);
-      uint32_t s1 = 0, p1 = 0, s2 = 0, p2 = 0, rph = 0;
-      int c1_last[C::ST1], c2_last[C::ST2], r_last = -1;
-      for (int s = 0; s < C::ST1; ++s) c1_last[s] = -1;
-      for (int s = 0; s < C::ST2; ++s) c2_last[s] = -1;
-      bool ok = true;
-      uint32_t ist = 0, iph = 0;
-      int claimed = -1;
-      // Bulk zero fill: one unit per work item, claimed one item ahead so
-      // that the atomic's latency is not waited for.
-      const long long fill_units = bulk_fill ? static_cast<long long>(B) * H * fill_parts : 0;
-      int fill_u = -1;
-      auto issue_fill = [&]() {
-        if constexpr (C::ZBUF > 0) {
-          if (fill_u >= 0 && fill_u < fill_units) {
-            const FillRange f = zero_fill_range(fill_lengths, H, L, D, C::BM, fill_parts, fill_u);
-            uint8_t* g = reinterpret_cast<uint8_t*>(out1 + f.base);
-            constexpr long long kPiece = C::ZBUF / 16;  // 16-byte chunks per bulk copy
-            for (long long c = f.begin; c < f.end; c += kPiece)
-              bulk_store(g + c * 16, sbase + C::OFF_Z, static_cast<uint32_t>(min(kPiece, f.end - c) * 16));
-            bulk_commit();
-          }
-        }
-      };
-      while (ok) {
-        const Item item = next_item(ws, claimed, count);
-        if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, ws, 200))) break;
-        if (item.n < 0) break;
-        const int n = item.n;
-        const int hd = PACKED ? item.bh % H : 0;
-        const int nb = ceil_div(n, C::BN);
-        if (fill_units > 0 && fill_u < fill_units) {
-          issue_fill();
-          fill_u = atomicAdd(ws + kHdrFill, 1);
-        }
-        if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, ws, 201))) break;
-        mbar_arrive_expect_tx(&bar.r_full, 2 * C::TILE_R);
-        for (int c = 0; c < D / 64; ++c) {
-          const int ry = rm.y(item, hd, item.blk * C::BM), rz = rm.z(item, item.blk * C::BM);
-          tma_load_3d(smem + C::OFF_R1 + c * C::BOX_R, &tm_r1, &bar.r_full, c * 64, ry, rz);
-          tma_load_3d(smem + C::OFF_R2 + c * C::BOX_R, &tm_r2, &bar.r_full, c * 64, ry, rz);
-        }
-        r_last = static_cast<int>(rph);
-        rph ^= 1;
-        for (int j = 0; j < nb; ++j) {
-          // Claim the CTA's next item two column blocks before this one ends.
-          if (j == max(0, nb - 2)) claimed = atomicAdd(ws + kHdrNext, 1);
-          if (!(ok = mbar_wait(&bar.c1_empty[s1], p1 ^ 1, abort_flag, ws, 202))) break;
-          mbar_arrive_expect_tx(&bar.c1_full[s1], C::TILE_C);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + C::OFF_C1 + s1 * C::TILE_C + c * C::BOX_C, &tm_c1, &bar.c1_full[s1], c * 64,
-                        rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
-          c1_last[s1] = static_cast<int>(p1);
-          if (++s1 == C::ST1) { s1 = 0; p1 ^= 1; }
-          if (!(ok = mbar_wait(&bar.c2_empty[s2], p2 ^ 1, abort_flag, ws, 203))) break;
-          mbar_arrive_expect_tx(&bar.c2_full[s2], C::TILE_C);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + C::OFF_C2 + s2 * C::TILE_C + c * C::BOX_C, &tm_c2, &bar.c2_full[s2], c * 64,
-                        rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
-          c2_last[s2] = static_cast<int>(p2);
-          if (++s2 == C::ST2) { s2 = 0; p2 ^= 1; }
-        }
-      }
-      // The last unit claimed, then every bulk copy must have landed before
-      // the shared-memory zeros go away with the CTA.
-      if (fill_units > 0) {
-        issue_fill();
-        bulk_wait_all();
-      }
-      if (!ok) {  // aborting: let the copies in flight land before the CTA exits
-        int never = 0;
-        volatile int* no_abort = &never;
-        for (int s = 0; s < C::ST1; ++s)
-          if (c1_last[s] >= 0) mbar_wait(&bar.c1_full[s], c1_last[s], no_abort, nullptr, 0);
-        for (int s = 0; s < C::ST2; ++s)
-          if (c2_last[s] >= 0) mbar_wait(&bar.c2_full[s], c2_last[s], no_abort, nullptr, 0);
-        if (r_last >= 0) mbar_wait(&bar.r_full, r_last, no_abort, nullptr, 0);
-      }
-    }
-  } else if (warp == kSWarp || warp == kDPWarp) {
-    // ------------------------------------------ issuers of S = R1 C1^T, dP = R2 C2^T
-    if (lane == 0) {
-      const bool is_dp = (warp == kDPWarp);
-      constexpr uint32_t idesc_x = idesc_bf16_f32(128, C::BN, false, false);
-      const uint64_t d_r = smem_desc_sw128(sbase + (is_dp ? C::OFF_R2 : C::OFF_R1), 16, 1024);
-      const uint64_t d_c = smem_desc_sw128(sbase + (is_dp ? C::OFF_C2 : C::OFF_C1), 16, 1024);
-      const int nbuf = is_dp ? C::NXDP : 1;     // regions this issuer rotates through
-      const int slots = is_dp ? C::ST2 : C::ST1;
-      uint64_t* cfull = is_dp ? bar.c2_full : bar.c1_full;
-      uint64_t* cempty = is_dp ? bar.c2_empty : bar.c1_empty;
-      uint32_t st = 0, cph = 0, rph = 0, xb = 0;
-      uint32_t read_ph[2] = {0, 0};
-      bool ok = true;
-      uint32_t ist = 0, iph = 0;
-      while (ok) {
-        Item item;
-        if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 210))) break;
-        ring_release(bar.ring, ist, iph, true);
-        if (item.n < 0) break;
-        const int n = item.n;
-        const int nb = ceil_div(n, C::BN);
-        if (!(ok = mbar_wait(&bar.r_full, rph, abort_flag, ws, 211))) break;
-        rph ^= 1;
-        for (int j = 0; j < nb; ++j) {
-          if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 212))) break;
-          // The region is free once the epilogue has copied out the block that
-          // last used it (block j-1, or j-2 with two dP regions).
-          uint64_t* xread = is_dp ? &bar.xdp_read[xb] : &bar.xs_read;
-          uint64_t* xfull = is_dp ? &bar.xdp_full[xb] : &bar.xs_full;
-          const uint32_t d_tmem = tmem + (is_dp ? (xb ? C::TM_XDP1 : C::TM_XDP) : C::TM_XS);
-          if (!(ok = mbar_wait(xread, read_ph[xb] ^ 1, abort_flag, ws, 213))) break;
-          read_ph[xb] ^= 1;
-          tc_fence_after();
-          const uint64_t b0 = d_c + st * kTileC;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {  // K = D in steps of 16
-            const uint64_t a_off = ((kk >> 2) * C::BOX_R + (kk & 3) * 32) >> 4;
-            const uint64_t b_off = ((kk >> 2) * C::BOX_C + (kk & 3) * 32) >> 4;
-            mma_ss(d_tmem, d_r + a_off, b0 + b_off, idesc_x, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(xfull);
-          mma_commit(&cempty[st]);
-          if (++st == slots) { st = 0; cph ^= 1; }
-          if (++xb == static_cast<uint32_t>(nbuf)) xb = 0;
-          if (j + 1 == nb) mma_commit(&bar.r_empty);
-        }
-      }
-      int never = 0;
-      mma_commit(&bar.drain[is_dp ? 1 : 0]);
-      mbar_wait(&bar.drain[is_dp ? 1 : 0], 0, &never, ws, 219);
-    }
-  } else if (warp == kA1Warp || warp == kA2Warp) {
-    // -------------------------- issuers of A1 += dS C1 and (dK/dV) A2 += P C2
-    if (lane == 0) {
-      const bool second = (warp == kA2Warp);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
-      // MN-major view of the C1 (A1) or C2 (A2) ring: rows = the K dimension,
-      // the two 64-column halves of D BOX_C bytes apart.
-      const uint64_t d_cmn = smem_desc_sw128(sbase + (second ? C::OFF_C2 : C::OFF_C1), C::BOX_C, 1024);
-      const int slots = second ? C::ST2 : C::ST1;
-      uint64_t* cfull = second ? bar.c2_full : bar.c1_full;
-      uint64_t* cempty = second ? bar.c2_empty : bar.c1_empty;
-      const uint32_t tm_acc = tmem + (second ? C::TM_A2 : C::TM_A1);
-      const uint32_t tm_a = tmem + (second ? C::TM_P : C::TM_DS);
-      uint64_t* full = second ? bar.p_full : bar.ds_full;
-      uint64_t* freed = second ? &bar.p_free : &bar.ds_free;
-      uint32_t st = 0, cph = 0, aph = 0;
-      uint32_t fph[4] = {0, 0, 0, 0};
-      bool ok = true;
-      uint32_t ist = 0, iph = 0;
-      while (ok) {
-        Item item;
-        if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 210))) break;
-        ring_release(bar.ring, ist, iph, true);
-        if (item.n < 0) break;
-        const int n = item.n;
-        const int nb = ceil_div(n, C::BN);
-        for (int j = 0; ok && j < nb; ++j) {
-          if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 231))) break;
-          const uint64_t b0 = d_cmn + st * kTileC;
-          for (int q = 0; q < C::NCH; ++q) {
-            if (!(ok = mbar_wait(&full[q], fph[q], abort_flag, ws, 232))) break;
-            fph[q] ^= 1;
-            const bool first = (j == 0 && q == 0);
-            if (first) {
-              if (!(ok = mbar_wait(&bar.acc_empty, aph ^ 1, abort_flag, ws, 233))) break;
-              aph ^= 1;
-            }
-            tc_fence_after();
-            // K = the chunk's 32 columns: two K=16 steps; the chunk's bf16
-            // values sit in 16 TMEM columns (two per column).
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              mma_ts(tm_acc, tm_a + q * 16 + kk * 8, b0 + ((q * 32 * 128 + kk * 2048) >> 4), idesc_acc,
-                     (first && kk == 0) ? 0u : 1u);
-          }
-          if (!ok) break;
-          mma_commit(freed);
-          mma_commit(&cempty[st]);
-          if (++st == slots) { st = 0; cph ^= 1; }
-        }
-        if (!ok) break;
-        mma_commit(&bar.acc_full);
-      }
-      int never = 0;
-      mma_commit(&bar.drain[second ? 3 : 2]);
-      mbar_wait(&bar.drain[second ? 3 : 2], 0, &never, ws, 239);
-    }
-  } else if (warp < C::EPI_WARPS) {
+  if (warp < C::EPI_WARPS) {
     // ------------------------------------------------------------- epilogue
+    setmaxnreg_inc<C::EPI_REGS>();
     constexpr int CPW = C::CPW;
     const int g = warp >> 2;                      // chunks g*CPW .. g*CPW + CPW - 1
     const int r = ((warp & 3) << 5) + lane;       // row within the item = TMEM lane
@@ -383,7 +206,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     const uint32_t tXDP0 = tmem + lane_off + C::TM_XDP + g * CPW * 32;
     const uint32_t tXDP1 = tmem + lane_off + C::TM_XDP1 + g * CPW * 32;
     constexpr float scale = Scale<D>::value;
-    const uint64_t scale_l2e2 = f2_splat(scale * kLog2e);
+    constexpr float scale_l2e = scale * kLog2e;
     uint32_t s_ph = 0, free_ph = 0, aph = 0, xb = 0;
     uint32_t dp_ph[2] = {0, 0};
     bool ok = true;
@@ -395,14 +218,16 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       ring_release(bar.ring, ist, iph, lane == 0);
       if (item.n < 0) break;
       const int n = item.n;
-      const int nb = ceil_div(n, C::BN);
-      const uint64_t neg_log2n2 = f2_splat(-__log2f(static_cast<float>(n)));  // bias * log2(e)
+      const int ncols = work_cols(KV ? kKindDkdv : kKindDq, n, kr);
+      const int nb = ceil_div(ncols, C::BN);
+      const bool row_ok = item.blk * C::BM + r < (KV ? range_keys(n, kr) : n);  // this lane's row is a valid token
+      const float neg_log2n = -__log2f(static_cast<float>(n));  // bias * log2(e)
       for (int j = 0; j < nb; ++j) {
         // ---- S -> sigma'(x) = P (1 - P) kept in registers for dS, and (dK/dV)
         // bf16 P for dV, stored chunk by chunk as it is computed (the P region
         // is free once the previous block's dV products have read it). Padded
         // columns get P = sigma' = 0.
-        uint64_t sp[CPW][16];  // sigma' of column pairs (2e, 2e + 1)
+        float sp[CPW][32];
         {
           uint32_t sv[CPW][32];
           if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, ws, 221))) break;
@@ -419,25 +244,15 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
             if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
             tc_fence_after();
           }
-          const int valid = n - (j * C::BN + g * CPW * 32);  // columns < valid are real tokens
+          const int valid = ncols - (j * C::BN + g * CPW * 32);  // columns < valid are real tokens
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
             uint32_t pk[16];
+            mask_scores(sv[c], valid - 32 * c, row_ok);
+            sigmoid32<true>(sv[c], scale_l2e, neg_log2n, sp[c]);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              uint64_t slope;
-              const uint64_t pp = sigmoid2<true>(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1]),
-                                                 scale_l2e2, neg_log2n2, &slope);
-              if (valid < CPW * 32) {
-                const float2 p = f2_unpack(pp), d = f2_unpack(slope);
-                const bool v0 = 32 * c + 2 * e < valid, v1 = 32 * c + 2 * e + 1 < valid;
-                pk[e] = pack_bf16x2(v0 ? p.x : 0.f, v1 ? p.y : 0.f);
-                sp[c][e] = f2_pack(v0 ? d.x : 0.f, v1 ? d.y : 0.f);
-              } else {
-                pk[e] = pack_bf16x2_pair(pp);
-                sp[c][e] = slope;
-              }
-            }
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1]));
             if (KV) {
               tmem_st16(tmem + lane_off + C::TM_P + (g * CPW + c) * 16, pk);
               tmem_st_wait();
@@ -483,8 +298,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           uint32_t dk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            dk[e] = pack_bf16x2_pair(f2_mul(f2_pack(__uint_as_float(dpc[2 * e]), __uint_as_float(dpc[2 * e + 1])),
-                                            sp[c][e]));
+            dk[e] = pack_bf16x2(__uint_as_float(dpc[2 * e]) * sp[c][2 * e],
+                                __uint_as_float(dpc[2 * e + 1]) * sp[c][2 * e + 1]);
           tmem_st16(tmem + lane_off + C::TM_DS + (g * CPW + c) * 16, dk);
           tmem_st_wait();
           tc_fence_before();
@@ -498,7 +313,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       tc_fence_after();
       const int row = item.blk * C::BM + r;
       const bool in_range = rm.writes(row, n);
-      const bool valid_row = row < n;
+      const bool valid_row = row < (KV ? range_keys(n, kr) : n);
       const size_t row_off = rm.offset(item, PACKED ? item.bh % H : 0, row, D);
       // 32-column chunks of the accumulators: A1 (-> out1, times scale), then
       // A2 (-> out2) for dK/dV; each half of the warps takes every other
@@ -506,7 +321,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       // accumulators are released before the (slower) global stores.
       constexpr int kChunks = (KV ? 2 : 1) * (D / 32);
       constexpr int kPer = kChunks / 2;
-      uint32_t packed[kPer][16];
+      // bf16 pairs, or (F32OUT) the fp32 values themselves
+      uint32_t packed[kPer][F32OUT ? 32 : 16];
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
         const int c = g + 2 * i;
@@ -515,9 +331,14 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         const float mul = (second ? 1.0f : scale) * (valid_row ? 1.0f : 0.0f);
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v);
+        if constexpr (F32OUT) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          packed[i][e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+          for (int e = 0; e < 32; ++e) packed[i][e] = valid_row ? __float_as_uint(__uint_as_float(v[e]) * mul) : 0u;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            packed[i][e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -528,28 +349,232 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const int c = g + 2 * i;
           const bool second = c >= D / 32;
           const int col = (second ? c - D / 32 : c) * 32;
-          if (valid_row) {
-            store_row64B((second ? out2 : out1) + row_off + col, packed[i]);
+          void* out = second ? out2 : out1;
+          if constexpr (F32OUT) {
+            store_row_f32(static_cast<float*>(out) + row_off + col, packed[i]);  // zeros already for padded rows
+          } else if (valid_row) {
+            store_row64B(static_cast<__nv_bfloat16*>(out) + row_off + col, packed[i]);
           } else {
-            store_zero32((second ? out2 : out1) + row_off + col);
+            store_zero32(static_cast<__nv_bfloat16*>(out) + row_off + col);
           }
         }
       }
     }
+  } else {
+    // The producer, the issuers and the idle warps (one warpgroup pair) hand
+    // registers to the epilogue.
+    setmaxnreg_dec<C::OTHER_REGS>();
+    if (warp == kProducerWarp) {
+      // ------------------------------------------------------------- producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_r1);
+        tma_prefetch_desc(&tm_r2);
+        tma_prefetch_desc(&tm_c1);
+        tma_prefetch_desc(&tm_c2);
+        uint32_t s1 = 0, p1 = 0, s2 = 0, p2 = 0, rph = 0;
+        int c1_last[C::ST1], c2_last[C::ST2], r_last = -1;
+        for (int s = 0; s < C::ST1; ++s) c1_last[s] = -1;
+        for (int s = 0; s < C::ST2; ++s) c2_last[s] = -1;
+        bool ok = true;
+        uint32_t ist = 0, iph = 0;
+        int claimed = -1;
+        // Bulk zero fill: one unit per work item, claimed one item ahead so
+        // that the atomic's latency is not waited for.
+        const long long fill_units = bulk_fill ? static_cast<long long>(B) * H * fill_parts : 0;
+        int fill_u = -1;
+        auto issue_fill = [&]() {
+          if constexpr (C::ZBUF > 0) {
+            if (fill_u >= 0 && fill_u < fill_units) {
+              const FillRange f = zero_fill_range(fill_lengths, fill_geom, fill_parts, fill_u);
+              uint8_t* g = reinterpret_cast<uint8_t*>(out1) + f.base * 16;
+              constexpr long long kPiece = C::ZBUF / 16;  // 16-byte chunks per bulk copy
+              for (long long c = f.begin; c < f.end; c += kPiece)
+                bulk_store(g + c * 16, sbase + C::OFF_Z, static_cast<uint32_t>(min(kPiece, f.end - c) * 16));
+              bulk_commit();
+            }
+          }
+        };
+        while (ok) {
+          const Item item = next_item(ws, claimed, count);
+          if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, ws, 200))) break;
+          if (item.n < 0) break;
+          const int n = item.n;
+          const int hd = PACKED ? item.bh % H : 0;
+          const int nb = ceil_div(work_cols(KV ? kKindDkdv : kKindDq, n, kr), C::BN);
+          if (fill_units > 0 && fill_u < fill_units) {
+            issue_fill();
+            fill_u = atomicAdd(ws + kHdrFill, 1);
+          }
+          if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, ws, 201))) break;
+          mbar_arrive_expect_tx(&bar.r_full, 2 * C::TILE_R);
+          for (int c = 0; c < D / 64; ++c) {
+            const int ry = rm.y(item, hd, item.blk * C::BM), rz = rm.z(item, item.blk * C::BM);
+            tma_load_3d(smem + C::OFF_R1 + c * C::BOX_R, &tm_r1, &bar.r_full, c * 64, ry, rz);
+            tma_load_3d(smem + C::OFF_R2 + c * C::BOX_R, &tm_r2, &bar.r_full, c * 64, ry, rz);
+          }
+          r_last = static_cast<int>(rph);
+          rph ^= 1;
+          for (int j = 0; j < nb; ++j) {
+            // Claim the CTA's next item two column blocks before this one ends.
+            if (j == max(0, nb - 2)) claimed = atomicAdd(ws + kHdrNext, 1);
+            if (!(ok = mbar_wait(&bar.c1_empty[s1], p1 ^ 1, abort_flag, ws, 202))) break;
+            mbar_arrive_expect_tx(&bar.c1_full[s1], C::TILE_C);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(smem + C::OFF_C1 + s1 * C::TILE_C + c * C::BOX_C, &tm_c1, &bar.c1_full[s1], c * 64,
+                          rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
+            c1_last[s1] = static_cast<int>(p1);
+            if (++s1 == C::ST1) { s1 = 0; p1 ^= 1; }
+            if (!(ok = mbar_wait(&bar.c2_empty[s2], p2 ^ 1, abort_flag, ws, 203))) break;
+            mbar_arrive_expect_tx(&bar.c2_full[s2], C::TILE_C);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(smem + C::OFF_C2 + s2 * C::TILE_C + c * C::BOX_C, &tm_c2, &bar.c2_full[s2], c * 64,
+                          rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
+            c2_last[s2] = static_cast<int>(p2);
+            if (++s2 == C::ST2) { s2 = 0; p2 ^= 1; }
+          }
+        }
+        // The last unit claimed, then every bulk copy must have landed before
+        // the shared-memory zeros go away with the CTA.
+        if (fill_units > 0) {
+          issue_fill();
+          bulk_wait_all();
+        }
+        if (!ok) {  // aborting: let the copies in flight land before the CTA exits
+          int never = 0;
+          volatile int* no_abort = &never;
+          for (int s = 0; s < C::ST1; ++s)
+            if (c1_last[s] >= 0) mbar_wait(&bar.c1_full[s], c1_last[s], no_abort, nullptr, 0);
+          for (int s = 0; s < C::ST2; ++s)
+            if (c2_last[s] >= 0) mbar_wait(&bar.c2_full[s], c2_last[s], no_abort, nullptr, 0);
+          if (r_last >= 0) mbar_wait(&bar.r_full, r_last, no_abort, nullptr, 0);
+        }
+      }
+    } else if (warp == kSWarp || warp == kDPWarp) {
+      // ------------------------------------------ issuers of S = R1 C1^T, dP = R2 C2^T
+      if (lane == 0) {
+        const bool is_dp = (warp == kDPWarp);
+        constexpr uint32_t idesc_x = idesc_bf16_f32(128, C::BN, false, false);
+        const uint64_t d_r = smem_desc_sw128(sbase + (is_dp ? C::OFF_R2 : C::OFF_R1), 16, 1024);
+        const uint64_t d_c = smem_desc_sw128(sbase + (is_dp ? C::OFF_C2 : C::OFF_C1), 16, 1024);
+        const int nbuf = is_dp ? C::NXDP : 1;     // regions this issuer rotates through
+        const int slots = is_dp ? C::ST2 : C::ST1;
+        uint64_t* cfull = is_dp ? bar.c2_full : bar.c1_full;
+        uint64_t* cempty = is_dp ? bar.c2_empty : bar.c1_empty;
+        uint32_t st = 0, cph = 0, rph = 0, xb = 0;
+        uint32_t read_ph[2] = {0, 0};
+        bool ok = true;
+        uint32_t ist = 0, iph = 0;
+        while (ok) {
+          Item item;
+          if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 210))) break;
+          ring_release(bar.ring, ist, iph, true);
+          if (item.n < 0) break;
+          const int n = item.n;
+          const int nb = ceil_div(work_cols(KV ? kKindDkdv : kKindDq, n, kr), C::BN);
+          if (!(ok = mbar_wait(&bar.r_full, rph, abort_flag, ws, 211))) break;
+          rph ^= 1;
+          for (int j = 0; j < nb; ++j) {
+            if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 212))) break;
+            // The region is free once the epilogue has copied out the block that
+            // last used it (block j-1, or j-2 with two dP regions).
+            uint64_t* xread = is_dp ? &bar.xdp_read[xb] : &bar.xs_read;
+            uint64_t* xfull = is_dp ? &bar.xdp_full[xb] : &bar.xs_full;
+            const uint32_t d_tmem = tmem + (is_dp ? (xb ? C::TM_XDP1 : C::TM_XDP) : C::TM_XS);
+            if (!(ok = mbar_wait(xread, read_ph[xb] ^ 1, abort_flag, ws, 213))) break;
+            read_ph[xb] ^= 1;
+            tc_fence_after();
+            const uint64_t b0 = d_c + st * kTileC;
+  #pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {  // K = D in steps of 16
+              const uint64_t a_off = ((kk >> 2) * C::BOX_R + (kk & 3) * 32) >> 4;
+              const uint64_t b_off = ((kk >> 2) * C::BOX_C + (kk & 3) * 32) >> 4;
+              mma_ss(d_tmem, d_r + a_off, b0 + b_off, idesc_x, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(xfull);
+            mma_commit(&cempty[st]);
+            if (++st == slots) { st = 0; cph ^= 1; }
+            if (++xb == static_cast<uint32_t>(nbuf)) xb = 0;
+            if (j + 1 == nb) mma_commit(&bar.r_empty);
+          }
+        }
+        int never = 0;
+        mma_commit(&bar.drain[is_dp ? 1 : 0]);
+        mbar_wait(&bar.drain[is_dp ? 1 : 0], 0, &never, ws, 219);
+      }
+    } else if (warp == kA1Warp || warp == kA2Warp) {
+      // -------------------------- issuers of A1 += dS C1 and (dK/dV) A2 += P C2
+      if (lane == 0) {
+        const bool second = (warp == kA2Warp);
+        constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+        // MN-major view of the C1 (A1) or C2 (A2) ring: rows = the K dimension,
+        // the two 64-column halves of D BOX_C bytes apart.
+        const uint64_t d_cmn = smem_desc_sw128(sbase + (second ? C::OFF_C2 : C::OFF_C1), C::BOX_C, 1024);
+        const int slots = second ? C::ST2 : C::ST1;
+        uint64_t* cfull = second ? bar.c2_full : bar.c1_full;
+        uint64_t* cempty = second ? bar.c2_empty : bar.c1_empty;
+        const uint32_t tm_acc = tmem + (second ? C::TM_A2 : C::TM_A1);
+        const uint32_t tm_a = tmem + (second ? C::TM_P : C::TM_DS);
+        uint64_t* full = second ? bar.p_full : bar.ds_full;
+        uint64_t* freed = second ? &bar.p_free : &bar.ds_free;
+        uint32_t st = 0, cph = 0, aph = 0;
+        uint32_t fph[4] = {0, 0, 0, 0};
+        bool ok = true;
+        uint32_t ist = 0, iph = 0;
+        while (ok) {
+          Item item;
+          if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 210))) break;
+          ring_release(bar.ring, ist, iph, true);
+          if (item.n < 0) break;
+          const int n = item.n;
+          const int nb = ceil_div(work_cols(KV ? kKindDkdv : kKindDq, n, kr), C::BN);
+          for (int j = 0; ok && j < nb; ++j) {
+            if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 231))) break;
+            const uint64_t b0 = d_cmn + st * kTileC;
+            for (int q = 0; q < C::NCH; ++q) {
+              if (!(ok = mbar_wait(&full[q], fph[q], abort_flag, ws, 232))) break;
+              fph[q] ^= 1;
+              const bool first = (j == 0 && q == 0);
+              if (first) {
+                if (!(ok = mbar_wait(&bar.acc_empty, aph ^ 1, abort_flag, ws, 233))) break;
+                aph ^= 1;
+              }
+              tc_fence_after();
+              // K = the chunk's 32 columns: two K=16 steps; the chunk's bf16
+              // values sit in 16 TMEM columns (two per column).
+  #pragma unroll
+              for (int kk = 0; kk < 2; ++kk)
+                mma_ts(tm_acc, tm_a + q * 16 + kk * 8, b0 + ((q * 32 * 128 + kk * 2048) >> 4), idesc_acc,
+                       (first && kk == 0) ? 0u : 1u);
+            }
+            if (!ok) break;
+            mma_commit(freed);
+            mma_commit(&cempty[st]);
+            if (++st == slots) { st = 0; cph ^= 1; }
+          }
+          if (!ok) break;
+          mma_commit(&bar.acc_full);
+        }
+        int never = 0;
+        mma_commit(&bar.drain[second ? 3 : 2]);
+        mbar_wait(&bar.drain[second ? 3 : 2], 0, &never, ws, 239);
+      }
+    }
   }
 
-  // dQ over padded inputs: the fill units the producer did not take (all of
-  // them at D = 128, which has no room for the zeros in shared memory) are
-  // zeroed here, in the kernel's tail. Each warp joins once its role is done
-  // and claims units from the same workspace counter.
-  if (!KV && fill_lengths != nullptr) {
+  // Padded inputs: the output rows no item covers are zeroed by the warps
+  // without a role from the start (they come straight here) and by every other
+  // warp once its role is done, claiming fill units from the workspace counter
+  // that the dQ kernel's producer also takes units from for its bulk copies.
+  if (fill_lengths != nullptr) {
     const long long units = static_cast<long long>(B) * H * fill_parts;
     while (true) {
       int u = 0;
       if (lane == 0) u = atomicAdd(ws + kHdrFill, 1);
       u = __shfl_sync(0xffffffffu, u, 0);
       if (u >= units) break;
-      zero_fill_range_warp(zero_fill_range(fill_lengths, H, L, D, C::BM, fill_parts, u), lane, out1);
+      const FillRange f = zero_fill_range(fill_lengths, fill_geom, fill_parts, u);
+      zero_fill_range_warp(f, lane, out1);
+      if (KV) zero_fill_range_warp(f, lane, out2);
     }
   }
 
@@ -561,51 +586,70 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   }
 }
 
-template <int D, bool KV, bool PACKED>
+template <int D, bool KV, bool PACKED, bool F32OUT>
 cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
-                            const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
-                            const int* fill_lengths, cudaStream_t stream) {
+                            const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, KeyRange kr,
+                            int num_sms, const int* fill_lengths, int len_bound, cudaStream_t stream) {
   using C = BwdCfg<D, KV>;
   static PerDeviceOnce attr;
   const cudaError_t e = attr.run([] {
-    return cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED, F32OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 C::SMEM_ALLOC);
   });
   if (e != cudaSuccess) return e;
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kBwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
   const int parts = zero_fill_parts(static_cast<long long>(B) * H, num_sms);
-  return launch_programmatic(bwd_kernel<D, KV, PACKED>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, r1, r2,
-                             c1, c2, static_cast<__nv_bfloat16*>(out1), static_cast<__nv_bfloat16*>(out2), ws, H, L,
-                             fill_lengths, B, parts);
+  return launch_programmatic(bwd_kernel<D, KV, PACKED, F32OUT>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream,
+                             r1, r2, c1, c2, out1, out2, ws, H, L, kr, fill_lengths, B, len_bound, parts);
 }
 
-template <bool KV>
-cudaError_t launch_bwd(int d, bool packed, const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
-                       const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, int num_sms,
-                       const int* fill_lengths, cudaStream_t stream) {
+// fill_lengths: the padded layout's lengths, so that the kernel zeroes the
+// output rows no item covers itself (nullptr for the packed layout, whose
+// calls write only the rows of the sequences). kr: the keys the call covers
+// ({0, L} for whole sequences); f32out: dQ as the fp32 partial sum over them.
+cudaError_t launch_bwd_dq(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tdo,
+                          const CUtensorMap& tk, const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L,
+                          KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream) {
   if (packed) {
     if (d == 64)
-      return launch_bwd_impl<64, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
-    return launch_bwd_impl<128, KV, true>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, nullptr, stream);
+      return launch_bwd_impl<64, false, true, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms, nullptr,
+                                                     L, stream);
+    return launch_bwd_impl<128, false, true, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms, nullptr,
+                                                    L, stream);
+  }
+  if (f32out) {
+    if (d == 64)
+      return launch_bwd_impl<64, false, false, true>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms,
+                                                     fill_lengths, L, stream);
+    return launch_bwd_impl<128, false, false, true>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms,
+                                                    fill_lengths, L, stream);
   }
   if (d == 64)
-    return launch_bwd_impl<64, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
-  return launch_bwd_impl<128, KV, false>(r1, r2, c1, c2, out1, out2, ws, B, H, L, num_sms, fill_lengths, stream);
+    return launch_bwd_impl<64, false, false, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms,
+                                                    fill_lengths, L, stream);
+  return launch_bwd_impl<128, false, false, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms,
+                                                   fill_lengths, L, stream);
 }
 
-// fill_lengths: the padded layout's lengths, so that the dQ kernel zeroes the
-// uncovered rows of dQ itself (nullptr for the packed layout).
-cudaError_t launch_bwd_dq(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                          const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L, int num_sms,
-                          const int* fill_lengths, cudaStream_t stream) {
-  return launch_bwd<false>(d, packed, tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, num_sms, fill_lengths, stream);
-}
-
+// out_rows: rows per (b, h) slice of dK and dV (Lmax, or kr.count for a key
+// range, whose K and V maps hold only the range's keys); Lmax bounds the valid
+// lengths.
 cudaError_t launch_bwd_dkdv(int d, bool packed, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                            const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int L, int num_sms,
-                            cudaStream_t stream) {
-  return launch_bwd<true>(d, packed, tk, tv, tq, tdo, dk, dv, ws, B, H, L, num_sms, nullptr, stream);
+                            const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int out_rows, int Lmax,
+                            KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream) {
+  if (packed) {
+    if (d == 64)
+      return launch_bwd_impl<64, true, true, false>(tk, tv, tq, tdo, dk, dv, ws, B, H, out_rows, kr, num_sms, nullptr,
+                                                    Lmax, stream);
+    return launch_bwd_impl<128, true, true, false>(tk, tv, tq, tdo, dk, dv, ws, B, H, out_rows, kr, num_sms, nullptr,
+                                                   Lmax, stream);
+  }
+  if (d == 64)
+    return launch_bwd_impl<64, true, false, false>(tk, tv, tq, tdo, dk, dv, ws, B, H, out_rows, kr, num_sms,
+                                                   fill_lengths, Lmax, stream);
+  return launch_bwd_impl<128, true, false, false>(tk, tv, tq, tdo, dk, dv, ws, B, H, out_rows, kr, num_sms,
+                                                  fill_lengths, Lmax, stream);
 }
 
 }  // namespace sigattn

@@ -43,6 +43,47 @@ __device__ __forceinline__ int load_len(const int* lengths, int b, int L) {
   return (n < 0 || n > L) ? 0 : n;
 }
 
+// The keys a call covers: positions [begin, begin + count) of every
+// sequence. The ordinary calls cover whole sequences ({0, Lmax}); a call over
+// a key range computes the contribution of those keys only (the partial sums
+// of a key-sharded forward and dQ; the dK/dV rows of those keys). The bias
+// -ln n_b always uses the sequence's full length n_b.
+struct KeyRange {
+  int begin, count;
+};
+
+// Valid keys of a sequence of n tokens inside the range.
+__host__ __device__ inline int range_keys(int n, KeyRange kr) {
+  return n - kr.begin < 0 ? 0 : (n - kr.begin > kr.count ? kr.count : n - kr.begin);
+}
+
+// Rows that get work items: forward/dQ all n query rows when the range holds
+// a valid key (none otherwise); dK/dV the range's valid keys.
+__host__ __device__ inline int work_rows(int kind, int n, KeyRange kr) {
+  const int nk = range_keys(n, kr);
+  return kind == kKindDkdv ? nk : (nk > 0 ? n : 0);
+}
+
+// Columns each item walks: forward/dQ the range's valid keys; dK/dV all n
+// queries. (For whole-sequence calls both are n.)
+__host__ __device__ inline int work_cols(int kind, int n, KeyRange kr) {
+  return kind == kKindDkdv ? n : range_keys(n, kr);
+}
+
+// Where a call's zero fill writes: rows [cover, out_rows) of every (b, h)
+// slice of an output with `chunks_per_row` 16-byte chunks per row, cover being
+// the rows its work items write (work_rows rounded up to whole items).
+struct FillGeom {
+  int H, L;            // heads; the bound on valid lengths (Lmax)
+  int out_rows;        // rows per slice of the output (Lmax, or the key range's count for dK/dV)
+  int chunks_per_row;  // d * element bytes / 16
+  int kind, item_rows;
+  KeyRange kr;
+  __device__ __forceinline__ int cover(int n) const {
+    return min(out_rows, ceil_div(work_rows(kind, n, kr), item_rows) * item_rows);
+  }
+};
+
 // One work item as the plan stores it: 16 bytes {b * H + h, row block, n_b,
 // start_b}, so a kernel learns the item, its sequence's valid length and (for
 // packed inputs) the sequence's first token from one load.
@@ -148,32 +189,34 @@ struct Scale<128> {
 // Training: Sigmoid Attention for single-cell Foundation Models, sec. 2A); the
 // kernels form y = x log2(e) = s * scale_l2e + neg_log2n in one FMA and take
 //
-//   u = 2^(-|y|) = e^(-|x|)              (ex2.approx, relative error ~1e-7)
-//   r = 1 - u + kR2 u^2 + kR3 u^3 + kR4 u^4  ~  1 / (1 + u) on [0, 1]
-//   q = u r ~ sigma(-|x|),   sigma(x) = q for x < 0, r for x >= 0,
-//   sigma'(x) = sigma(x) sigma(-x) = q r.
+//   u = 2^(-|y|) = e^(-|x|)                      (ex2.approx, relative error ~1e-7)
+//   t = -1 + kR2 u + kR3 u^2 + kR4 u^3,  r = 1 + u t  ~  1 / (1 + u) on [0, 1]
+//   q = u + (u t) u = u r  ~  sigma(-|x|)
+//   sigma(x) = q for x < 0, r for x >= 0;   sigma'(x) = sigma(x) sigma(-x) = q r.
 //
-// The polynomial keeps r(0) = 1 and r'(0) = -1 exactly, so the weights of the
-// far tail (the usual case: the bias puts typical weights near 1/n) carry a
-// relative error of ~1e-6, and r(1) = 1/2, so sigma(0) = 1/2 and sigma'(0) =
-// 1/4; a minimax fit of the other coefficients bounds the relative error of
-// sigma by 9e-4 over the whole line (largest near |x| = 1.5), below the bf16
-// rounding that P undergoes next.
+// r keeps r(0) = 1 and r'(0) = -1 exactly, so the weights of the far tail (the
+// usual case: the bias puts typical weights near 1/n) carry a relative error
+// of ~1e-6, and r(1) = 1/2, so sigma(0) = 1/2 and sigma'(0) = 1/4; a minimax
+// fit of the other coefficients bounds the relative error of sigma by 9e-4 over
+// the whole line (largest near |x| = 1.5), below the bf16 rounding that P
+// undergoes next.
 //
 // The pages' kernel takes sigma from the hardware tanh, 1/2 + tanh(x/2)/2
 // (sec. 2C). Measured on B200, that form's error is a few 1e-6 in absolute
 // terms, which near 1/n is a relative error of up to 1 % (x in [-12, -8]) and
 // which drops every weight below ~1e-7 to zero; with all weights of a row near
 // 1/n it shifts O by the same relative amount. The form here costs the same
-// single MUFU operation per score; its FMAs run two scores at a time on the
-// packed fp32x2 pipe of sm_100, so it adds about three issue slots per score.
+// single MUFU operation per score, plus FMAs; the choice between q and r runs
+// on the integer/logic pipe. A warp whose scores all lie in the far tail takes
+// a shorter form without |y|, the polynomial's upper terms or the choice
+// (sigmoid32 below).
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kR2 = 0.9339003266f;
 constexpr float kR3 = -0.6298789201f;
 constexpr float kR4 = 0.1959785935f;
 
-// Two fp32 values in one 64-bit register (low half = first), for the packed
-// fp32x2 arithmetic of sm_100 (one instruction per two values).
+// Two fp32 values in one 64-bit register (first value in the low half), for
+// the packed fp32x2 FMAs of sm_100 (one instruction per two values).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -184,10 +227,10 @@ __device__ __forceinline__ float2 f2_unpack(uint64_t v) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
   return r;
 }
-__host__ __device__ constexpr uint64_t f2_splat_bits(uint32_t bits) {
-  return (static_cast<uint64_t>(bits) << 32) | bits;
+__device__ __forceinline__ uint64_t f2_splat(float x) {
+  const uint64_t b = __float_as_uint(x);
+  return (b << 32) | b;
 }
-__device__ __forceinline__ uint64_t f2_splat(float x) { return f2_splat_bits(__float_as_uint(x)); }
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
@@ -199,52 +242,113 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return d;
 }
 
-// sigma of two scores (a, b) at once, as an fp32 pair; with `slope` also
-// sigma' of both. scale_l2e2 and neg_log2n2 are splat pairs of
-// scale * log2(e) and -log2(n).
+// t(u) of two values at once.
+__device__ __forceinline__ uint64_t poly_t2(uint64_t u) {
+  uint64_t t = f2_fma(f2_splat(kR4), u, f2_splat(kR3));
+  t = f2_fma(t, u, f2_splat(kR2));
+  return f2_fma(t, u, f2_splat(-1.0f));
+}
+
+// The far tail, y < kTailY (sigma < 0.06): with u = 2^y <= 1/16,
+// 1 / (1 + u) = 1 - u + u^2 - u^3/(1+u), so q = u (1 - u + u^2) has relative
+// error below u^3 <= 2.5e-4 (below 1e-6 once u < 0.01). The kernels evaluate
+// it from w = 2^(y + 4) = 16 u as q = w (c + w (-c^2 + c^3 w)), c = 1/16.
+constexpr float kTailY = -4.0f;
+constexpr float kTailC = 0.0625f;
+
+// sigma of 32 scores of one thread, in place: a[e] holds the fp32 bits of a
+// score on entry and of its weight on return; with SLOPE, slope[e] receives
+// sigma'. The branch is warp-uniform (every lane of the warp must call this
+// together, as the tcgen05 loads that feed it already require): when every
+// score of the warp lies in the far tail (the usual case once n is more than
+// about a thousand: the bias -ln n puts the typical weight near 1/n), the
+// short tail form serves; otherwise the general form. Pairs of columns
+// (2e, 2e + 1) go through the packed fp32x2 FMAs.
 template <bool SLOPE>
-__device__ __forceinline__ uint64_t sigmoid2(float a, float b, uint64_t scale_l2e2, uint64_t neg_log2n2,
-                                             uint64_t* slope) {
-  const float2 y = f2_unpack(f2_fma(f2_pack(a, b), scale_l2e2, neg_log2n2));
-  const uint64_t u = f2_pack(ex2_approx(-fabsf(y.x)), ex2_approx(-fabsf(y.y)));
-  uint64_t r = f2_fma(f2_splat(kR4), u, f2_splat(kR3));
-  r = f2_fma(r, u, f2_splat(kR2));
-  r = f2_fma(r, u, f2_splat(-1.0f));
-  r = f2_fma(r, u, f2_splat(1.0f));
-  const uint64_t q = f2_mul(u, r);
-  if (SLOPE) *slope = f2_mul(q, r);
-  const float2 qq = f2_unpack(q), rr = f2_unpack(r);
-  return f2_pack(y.x < 0.0f ? qq.x : rr.x, y.y < 0.0f ? qq.y : rr.y);
+__device__ __forceinline__ void sigmoid32(uint32_t (&a)[32], float scale_l2e, float neg_log2n, float* slope) {
+  const uint64_t c1 = f2_splat(scale_l2e), c0 = f2_splat(neg_log2n - kTailY);
+  uint64_t z[16];  // z = y - kTailY
+  uint32_t all = 0xffffffffu;  // AND of the words: bit 31 set iff every z < 0
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    z[e] = f2_fma(f2_pack(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1])), c1, c0);
+    all &= static_cast<uint32_t>(z[e]) & static_cast<uint32_t>(z[e] >> 32);
+  }
+  if (__all_sync(0xffffffffu, (all >> 31) != 0)) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float2 zz = f2_unpack(z[e]);
+      const uint64_t w = f2_pack(ex2_approx(zz.x), ex2_approx(zz.y));
+      uint64_t t = f2_fma(w, f2_splat(kTailC * kTailC * kTailC), f2_splat(-kTailC * kTailC));
+      t = f2_fma(t, w, f2_splat(kTailC));
+      const uint64_t q = f2_mul(t, w);
+      const float2 qq = f2_unpack(q);
+      if (SLOPE) {
+        const float2 sl = f2_unpack(f2_mul(q, f2_fma(q, f2_splat(-1.0f), f2_splat(1.0f))));  // q (1 - q)
+        slope[2 * e] = sl.x;
+        slope[2 * e + 1] = sl.y;
+      }
+      a[2 * e] = __float_as_uint(qq.x);
+      a[2 * e + 1] = __float_as_uint(qq.y);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float2 yy = f2_unpack(f2_fma(z[e], f2_splat(1.0f), f2_splat(kTailY)));
+      const uint64_t u = f2_pack(ex2_approx(-fabsf(yy.x)), ex2_approx(-fabsf(yy.y)));
+      const uint64_t t = poly_t2(u);
+      const uint64_t q = f2_fma(f2_mul(t, u), u, u);
+      const uint64_t r = f2_fma(t, u, f2_splat(1.0f));
+      const float2 qq = f2_unpack(q), rr = f2_unpack(r);
+      if (SLOPE) {
+        const float2 sl = f2_unpack(f2_mul(q, r));
+        slope[2 * e] = sl.x;
+        slope[2 * e + 1] = sl.y;
+      }
+      a[2 * e] = __float_as_uint(yy.x < 0.0f ? qq.x : rr.x);
+      a[2 * e + 1] = __float_as_uint(yy.y < 0.0f ? qq.y : rr.y);
+    }
+  }
 }
 
-// sigma of one score (the diagnostic entry point; the kernels use sigmoid2).
+// Scores that must not count: the columns at or past `valid` (keys beyond
+// the sequence) and every column of a row that is not a valid token. Set to
+// -inf, their weight and its derivative come out exactly 0 on either form,
+// and they take no part in the warp's choice of form, so values in padded
+// rows never change the bits of a valid output.
+__device__ __forceinline__ void mask_scores(uint32_t (&a)[32], int valid, bool row_ok) {
+  if (valid >= 32 && row_ok) return;
+#pragma unroll
+  for (int e = 0; e < 32; ++e)
+    if (!row_ok || e >= valid) a[e] = 0xff800000u;
+}
+
+// sigma (and sigma') of one score, as the kernels compute it (the diagnostic
+// entry point; its warp takes the tail form only when all 32 lanes' scores are
+// in the far tail).
 __device__ __forceinline__ float sigmoid_score(float s, float scale_l2e, float neg_log2n, float* slope) {
-  uint64_t sl = 0;
-  const float2 p = f2_unpack(sigmoid2<true>(s, s, f2_splat(scale_l2e), f2_splat(neg_log2n), &sl));
-  *slope = f2_unpack(sl).x;
-  return p.x;
-}
-
-// Pack an fp32 pair to a bf16x2 word (round to nearest even; first value low).
-__device__ __forceinline__ uint32_t pack_bf16x2_pair(uint64_t v) {
-  const float2 f = f2_unpack(v);
-  return pack_bf16x2(f.x, f.y);
+  uint32_t a[32];
+  float sl[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) a[e] = __float_as_uint(s);
+  sigmoid32<true>(a, scale_l2e, neg_log2n, sl);
+  *slope = sl[0];
+  return __uint_as_float(a[0]);
 }
 
 // Zero one unit of the output rows that no work item covers: rows
-// [ceil(n_b/rows)*rows, L) of slice u / parts are cut into `parts` interleaved
-// shares of 16-byte chunks, and this warp writes share u % parts of out0 (and
-// out1).
-__device__ __forceinline__ void zero_fill_unit(const int* lengths, int H, int L, int d, int rows, int parts,
-                                               long long u, int lane, __nv_bfloat16* out0, __nv_bfloat16* out1) {
+// [cover, out_rows) of slice u / parts (cover: the rows the call's items
+// write) are cut into `parts` interleaved shares of 16-byte chunks, and this
+// warp writes share u % parts of out0 (and out1).
+__device__ __forceinline__ void zero_fill_unit(const int* lengths, const FillGeom& g, int parts, long long u, int lane,
+                                               void* out0, void* out1) {
   const int slice = static_cast<int>(u / parts);
   const int part = static_cast<int>(u % parts);
-  const int n = load_len(lengths, slice / H, L);
-  const int cover = min(L, ceil_div(n, rows) * rows);
-  const long long nchunks = static_cast<long long>(L - cover) * (d / 8);  // 16-byte chunks
-  const size_t base = (static_cast<size_t>(slice) * L + cover) * d;
-  uint4* p0 = reinterpret_cast<uint4*>(out0 + base);
-  uint4* p1 = out1 ? reinterpret_cast<uint4*>(out1 + base) : nullptr;
+  const int cover = g.cover(load_len(lengths, slice / g.H, g.L));
+  const long long nchunks = static_cast<long long>(g.out_rows - cover) * g.chunks_per_row;
+  const size_t base = (static_cast<size_t>(slice) * g.out_rows + cover) * g.chunks_per_row;
+  uint4* p0 = reinterpret_cast<uint4*>(out0) + base;
+  uint4* p1 = out1 ? reinterpret_cast<uint4*>(out1) + base : nullptr;
   for (long long c = static_cast<long long>(part) * 32 + lane; c < nchunks; c += static_cast<long long>(parts) * 32) {
     p0[c] = make_uint4(0, 0, 0, 0);
     if (p1) p1[c] = make_uint4(0, 0, 0, 0);
@@ -253,30 +357,28 @@ __device__ __forceinline__ void zero_fill_unit(const int* lengths, int H, int L,
 
 // The same rows cut into `parts` consecutive shares instead (the dQ kernel's
 // fill, whose units go either to bulk copies or to warps): unit u covers the
-// 16-byte chunks [begin, end) counted from element `base` of the output.
+// 16-byte chunks [begin, end) counted from 16-byte chunk `base` of the output.
 struct FillRange {
   size_t base;
   long long begin, end;
 };
 
-__device__ __forceinline__ FillRange zero_fill_range(const int* lengths, int H, int L, int d, int rows, int parts,
-                                                     long long u) {
+__device__ __forceinline__ FillRange zero_fill_range(const int* lengths, const FillGeom& g, int parts, long long u) {
   const int slice = static_cast<int>(u / parts);
   const int part = static_cast<int>(u % parts);
-  const int n = load_len(lengths, slice / H, L);
-  const int cover = min(L, ceil_div(n, rows) * rows);
-  const long long nchunks = static_cast<long long>(L - cover) * (d / 8);
+  const int cover = g.cover(load_len(lengths, slice / g.H, g.L));
+  const long long nchunks = static_cast<long long>(g.out_rows - cover) * g.chunks_per_row;
   const long long share = (nchunks + parts - 1) / parts;
   FillRange f;
-  f.base = (static_cast<size_t>(slice) * L + cover) * d;
+  f.base = (static_cast<size_t>(slice) * g.out_rows + cover) * g.chunks_per_row;
   f.begin = min(nchunks, part * share);
   f.end = min(nchunks, f.begin + share);
   return f;
 }
 
 // One warp writes the zeros of a consecutive-share unit.
-__device__ __forceinline__ void zero_fill_range_warp(const FillRange& f, int lane, __nv_bfloat16* out) {
-  uint4* p = reinterpret_cast<uint4*>(out + f.base);
+__device__ __forceinline__ void zero_fill_range_warp(const FillRange& f, int lane, void* out) {
+  uint4* p = reinterpret_cast<uint4*>(out) + f.base;
   for (long long c = f.begin + lane; c < f.end; c += 32) p[c] = make_uint4(0, 0, 0, 0);
 }
 
@@ -337,6 +439,52 @@ struct PerDeviceOnce {
     return err[dev];
   }
 };
+
+// Store 32 fp32 values (one row's 32 columns, 128 bytes) at dst, 16-byte
+// aligned; 32-byte stores when dst is 32-byte aligned (warp-uniform).
+__device__ __forceinline__ void store_row_f32(float* dst, const uint32_t (&v)[32]) {
+  if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 8 * h), "r"(v[8 * h]),
+                   "r"(v[8 * h + 1]), "r"(v[8 * h + 2]), "r"(v[8 * h + 3]), "r"(v[8 * h + 4]), "r"(v[8 * h + 5]),
+                   "r"(v[8 * h + 6]), "r"(v[8 * h + 7])
+                   : "memory");
+  } else {
+    uint4* p = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) p[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  }
+}
+
+// An output row chunk of 32 columns at element offset `off` of `out`: bf16
+// (rounded, times `mul`) or, for the fp32 partial sums of a key-range call,
+// the fp32 values themselves (times `mul`). `zero` writes zeros instead.
+template <bool F32OUT>
+__device__ __forceinline__ void store_out32(void* out, size_t off, const uint32_t (&v)[32], float mul, bool zero) {
+  if constexpr (F32OUT) {
+    uint32_t w[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) w[e] = zero ? 0u : __float_as_uint(__uint_as_float(v[e]) * mul);
+    store_row_f32(static_cast<float*>(out) + off, w);
+  } else {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + off;
+    if (zero) store_zero32(dst);
+    else store_row32(dst, v, mul);
+  }
+}
+
+template <bool F32OUT>
+__device__ __forceinline__ void store_zero_out32(void* out, size_t off) {
+  if constexpr (F32OUT) {
+    uint32_t w[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) w[e] = 0u;
+    store_row_f32(static_cast<float*>(out) + off, w);
+  } else {
+    store_zero32(static_cast<__nv_bfloat16*>(out) + off);
+  }
+}
 
 // Launch `kernel` so that it may start while the previous kernel in `stream` is
 // still running (programmatic stream serialization). The kernel calls

@@ -81,11 +81,13 @@ struct FwdBarriers {
   int abort;
 };
 
-template <int D, bool PACKED>
+// F32OUT: the output is the fp32 partial sum over the call's key range (no
+// rounding to bf16), for key-range calls whose partial outputs are summed.
+template <int D, bool PACKED, bool F32OUT>
 __global__ void __launch_bounds__((16 + 3) * 32, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-               int* __restrict__ ws, int H, int L) {
+               const __grid_constant__ CUtensorMap tm_v, void* __restrict__ out, int* __restrict__ ws, int H, int L,
+               KeyRange kr) {
   using C = FwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ FwdBarriers<C::KST, C::VST> bar;
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
         const int hd = PACKED ? item.bh % H : 0;
         const int row0 = item.blk * (C::BM * C::NQ);
         const int ntiles = (row0 + C::BM < n) ? 2 : 1;
-        const int nkb = ceil_div(n, C::BN);
+        const int nkb = ceil_div(range_keys(n, kr), C::BN);  // K/V rows are the range's keys
         if (!(ok = mbar_wait(&bar.q_empty, qph ^ 1, abort_flag, ws, 101))) break;
         mbar_arrive_expect_tx(&bar.q_full, ntiles * C::TILE_BYTES);
         for (int t = 0; t < ntiles; ++t)
@@ -261,7 +263,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
         const int n = item.n;
         const int row0 = item.blk * (C::BM * C::NQ);
         const int ntiles = (row0 + C::BM < n) ? 2 : 1;
-        const int nkb = ceil_div(n, C::BN);
+        const int nkb = ceil_div(range_keys(n, kr), C::BN);
         if (t >= ntiles) {
           // Tile 1 is fully padded in this item. Its issuer issues nothing but
           // still waits for every load and gives its arrival on every shared
@@ -347,7 +349,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     const int r = ((warp & 3) << 5) + lane;        // row within a tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
     const int ot = c >> 1, oc = c & 1;
-    const uint64_t scale_l2e2 = f2_splat(Scale<D>::value * kLog2e);
+    constexpr float scale_l2e = Scale<D>::value * kLog2e;
     uint32_t sph[2] = {0, 0}, oph[2] = {0, 0}, pvph[2] = {0, 0};
     bool pv_pending[2] = {false, false};  // a P of the tile was written whose PV has not been awaited
     bool ok = true;
@@ -361,10 +363,11 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       const int n = item.n;
       const int row_base = item.blk * (C::BM * C::NQ);
       const int ntiles = (row_base + C::BM < n) ? 2 : 1;
-      const int nkb = ceil_div(n, C::BN);
-      const uint64_t neg_log2n2 = f2_splat(-__log2f(static_cast<float>(n)));  // bias * log2(e)
+      const int nk = range_keys(n, kr);
+      const int nkb = ceil_div(nk, C::BN);
+      const float neg_log2n = -__log2f(static_cast<float>(n));  // bias * log2(e)
       for (int j = 0; ok && j < nkb; ++j) {
-        const int valid = n - (j * C::BN + 32 * c);  // columns < valid are real keys
+        const int valid = nk - (j * C::BN + 32 * c);  // columns < valid are real keys
         for (int t = 0; t < ntiles; ++t) {
           if (!(ok = mbar_wait(&bar.s_full[t], sph[t], abort_flag, ws, 121))) break;
           sph[t] ^= 1;
@@ -375,17 +378,10 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.s_read[t]);
           uint32_t pk[16];
+          mask_scores(a, valid, row_base + t * C::BM + r < n);
+          sigmoid32<false>(a, scale_l2e, neg_log2n, nullptr);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t pp = sigmoid2<false>(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]), scale_l2e2,
-                                                neg_log2n2, nullptr);
-            if (valid < 32) {
-              const float2 p = f2_unpack(pp);
-              pk[e] = pack_bf16x2((2 * e < valid) ? p.x : 0.f, (2 * e + 1 < valid) ? p.y : 0.f);
-            } else {
-              pk[e] = pack_bf16x2_pair(pp);
-            }
-          }
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
           // The P region is free once the tile's previous PV products completed.
           if (pv_pending[t]) {
             if (!(ok = mbar_wait(&bar.pv_done[t], pvph[t], abort_flag, ws, 124))) break;
@@ -402,9 +398,9 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       }
       if (!ok) break;
       const int row = row_base + ot * C::BM + r;
-      __nv_bfloat16* orow = out + rm.offset(item, PACKED ? item.bh % H : 0, row, D) + 32 * oc;
+      const size_t orow = rm.offset(item, PACKED ? item.bh % H : 0, row, D) + 32 * oc;
       if (ot >= ntiles) {  // tile fully padded: its rows of O are zero (padded layout)
-        if (rm.writes(row, n)) store_zero32(orow);
+        if (rm.writes(row, n)) store_zero_out32<F32OUT>(out, orow);
         continue;
       }
       if (!(ok = mbar_wait(&bar.o_full[ot], oph[ot], abort_flag, ws, 122))) break;
@@ -415,10 +411,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.o_empty[ot]);
-      if (rm.writes(row, n)) {
-        if (row < n) store_row32(orow, v, 1.0f);
-        else store_zero32(orow);
-      }
+      if (rm.writes(row, n)) store_out32<F32OUT>(out, orow, v, 1.0f, row >= n);
     }
   } else {
     // ------------------------------------------------------------- epilogue
@@ -428,7 +421,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
     const uint32_t tS = tmem + lane_off + C::TM_S + t * 128 + h * 64;
     const uint32_t tO = tmem + lane_off + C::TM_O + t * D + h * (D / 2);
-    const uint64_t scale_l2e2 = f2_splat(Scale<D>::value * kLog2e);
+    constexpr float scale_l2e = Scale<D>::value * kLog2e;
     uint32_t sph = 0, oph = 0, turn_ph = 0;
     bool ok = true;
     uint32_t ist = 0, iph = 0;
@@ -442,16 +435,17 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       const bool two_tiles = item.blk * (C::BM * C::NQ) + C::BM < n;
       const int row0 = item.blk * (C::BM * C::NQ) + t * C::BM;
       const int row = row0 + r;
-      __nv_bfloat16* orow = out + rm.offset(item, PACKED ? item.bh % H : 0, row, D) + h * (D / 2);
+      const size_t orow = rm.offset(item, PACKED ? item.bh % H : 0, row, D) + h * (D / 2);
       if (row0 >= n) {  // tile fully padded: its rows of O are zero (padded layout)
         if (rm.writes(row, n)) {
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) store_zero32(orow + c * 32);
+          for (int c = 0; c < D / 64; ++c) store_zero_out32<F32OUT>(out, orow + c * 32);
         }
         continue;
       }
-      const int nkb = ceil_div(n, C::BN);
-      const uint64_t neg_log2n2 = f2_splat(-__log2f(static_cast<float>(n)));  // bias * log2(e)
+      const int nk = range_keys(n, kr);
+      const int nkb = ceil_div(nk, C::BN);
+      const float neg_log2n = -__log2f(static_cast<float>(n));  // bias * log2(e)
       for (int j = 0; j < nkb; ++j) {
         if (!(ok = mbar_wait(&bar.s_full[t], sph, abort_flag, ws, 121))) break;
         sph ^= 1;
@@ -462,7 +456,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           turn_ph ^= 1;
         }
         tc_fence_after();
-        const int valid = n - (j * C::BN + h * 64);  // columns < valid are real keys
+        const int valid = nk - (j * C::BN + h * 64);  // columns < valid are real keys
         // The half's 64 keys in two 32-column chunks; P of chunk c goes to
         // TMEM columns [16c, 16c + 16) of the half, which hold S values this
         // thread has already read (chunk 0's).
@@ -471,17 +465,10 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           uint32_t a[32];
           tmem_ld32(tS + 32 * c, a);
           uint32_t pk[16];
+          mask_scores(a, valid - 32 * c, row < n);
+          sigmoid32<false>(a, scale_l2e, neg_log2n, nullptr);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t pp = sigmoid2<false>(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]), scale_l2e2,
-                                                neg_log2n2, nullptr);
-            if (valid < 64) {
-              const float2 p = f2_unpack(pp);
-              pk[e] = pack_bf16x2((32 * c + 2 * e < valid) ? p.x : 0.f, (32 * c + 2 * e + 1 < valid) ? p.y : 0.f);
-            } else {
-              pk[e] = pack_bf16x2_pair(pp);
-            }
-          }
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
           tmem_st16(tS + 16 * c, pk);
         }
         tmem_st_wait();
@@ -509,10 +496,7 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       if (lane == 0) mbar_arrive(&bar.o_empty[t]);
       if (rm.writes(row, n)) {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          if (row < n) store_row32(orow + c * 32, v[c], 1.0f);
-          else store_zero32(orow + c * 32);
-        }
+        for (int c = 0; c < D / 64; ++c) store_out32<F32OUT>(out, orow + c * 32, v[c], 1.0f, row >= n);
       }
     }
   }
@@ -525,31 +509,38 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
   }
 }
 
-template <int D, bool PACKED>
+template <int D, bool PACKED, bool F32OUT>
 cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
-                            int B, int H, int L, int num_sms, cudaStream_t stream) {
+                            int B, int H, int L, KeyRange kr, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D>;
   static PerDeviceOnce attr;
   const cudaError_t e = attr.run([] {
-    return cudaFuncSetAttribute(fwd_kernel<D, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(fwd_kernel<D, PACKED, F32OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 C::SMEM_ALLOC);
   });
   if (e != cudaSuccess) return e;
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kFwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
-  return launch_programmatic(fwd_kernel<D, PACKED>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, tq, tk,
-                             tv, static_cast<__nv_bfloat16*>(o), ws, H, L);
+  return launch_programmatic(fwd_kernel<D, PACKED, F32OUT>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, tq,
+                             tk, tv, o, ws, H, L, kr);
 }
 
 // L is Lmax for the padded layout and the longest sequence for the packed one.
-cudaError_t launch_fwd(int d, bool packed, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       void* o, int* ws, int B, int H, int L, int num_sms, cudaStream_t stream) {
+// kr: the keys covered (whole sequences: {0, L}); f32out: write the fp32
+// partial sum over those keys (padded layout only).
+cudaError_t launch_fwd(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, void* o, int* ws, int B, int H, int L, KeyRange kr, int num_sms,
+                       cudaStream_t stream) {
   if (packed) {
-    if (d == 64) return launch_fwd_impl<64, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
-    return launch_fwd_impl<128, true>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+    if (d == 64) return launch_fwd_impl<64, true, false>(tq, tk, tv, o, ws, B, H, L, kr, num_sms, stream);
+    return launch_fwd_impl<128, true, false>(tq, tk, tv, o, ws, B, H, L, kr, num_sms, stream);
   }
-  if (d == 64) return launch_fwd_impl<64, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
-  return launch_fwd_impl<128, false>(tq, tk, tv, o, ws, B, H, L, num_sms, stream);
+  if (f32out) {
+    if (d == 64) return launch_fwd_impl<64, false, true>(tq, tk, tv, o, ws, B, H, L, kr, num_sms, stream);
+    return launch_fwd_impl<128, false, true>(tq, tk, tv, o, ws, B, H, L, kr, num_sms, stream);
+  }
+  if (d == 64) return launch_fwd_impl<64, false, false>(tq, tk, tv, o, ws, B, H, L, kr, num_sms, stream);
+  return launch_fwd_impl<128, false, false>(tq, tk, tv, o, ws, B, H, L, kr, num_sms, stream);
 }
 
 }  // namespace sigattn

@@ -12,14 +12,19 @@
 //     compute grid takes items round-robin, which spreads the long items over
 //     all SMs first (longest-processing-time-first order);
 //   * rows of the outputs that no item covers (rows >= ceil(n_b/rows)*rows)
-//     are written as exact zeros: after the forward and dK/dV kernels by
-//     fill_kernel, a one-warp-per-CTA kernel launched with a programmatic edge,
-//     so that it runs on the registers and warps the persistent compute CTA
-//     leaves free and its HBM writes overlap the compute-bound kernel; the dQ
-//     kernel zeroes its own: at d = 64 its producer issues bulk copies from a
-//     block of zeros in shared memory, one fill unit per work item, and in its
-//     tail each warp, once its role is done, claims the units left from the
-//     same counter in the workspace header.
+//     are written as exact zeros: after the forward kernel by fill_kernel, a
+//     one-warp-per-CTA kernel launched with a programmatic edge, so that it
+//     runs on the registers and warps the persistent compute CTA leaves free
+//     and its HBM writes overlap the compute-bound kernel; the backward
+//     kernels, whose CTAs take all of an SM's registers, zero their own: their
+//     warps without a role from the start and every other warp once its role
+//     is done claim fill units from a counter in the workspace header (at
+//     d = 64 the dQ kernel's producer also issues bulk copies from a block of
+//     zeros in shared memory, one fill unit per work item).
+//   * a call over a key range (a contiguous range of key positions of every
+//     sequence) enumerates the rows that have work: for the forward and dQ all
+//     query rows of a sequence with a valid key in the range, for dK/dV the
+//     range's valid keys; the items are ordered by their column counts.
 #include <algorithm>
 #include <numeric>
 #include <vector>
@@ -33,17 +38,19 @@ namespace sigattn {
 // [cu[b], cu[b+1]), which must lie inside [0, total_tokens]. A sequence that breaks
 // its bounds gets no work items and raises SIGATTN_ERR_INVALID_ARG.
 __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ lengths, const int* __restrict__ cu,
-                                                    int total_tokens, int B, int H, int L, int rows,
+                                                    int total_tokens, int B, int H, int L, int kind, KeyRange kr,
                                                     int* __restrict__ ws) {
   // The compute kernel that follows may set itself up meanwhile; it waits
   // for this grid before it reads the plan.
   grid_dep_launch();
   extern __shared__ int smem_plan[];
   const int tid = threadIdx.x;
+  const int rows = item_rows(kind);
   int* s_len = smem_plan;            // [B]
   int* s_order = smem_plan + B;      // [B]
   int* s_off = smem_plan + 2 * B;    // [B + 1]
   int* s_start = smem_plan + 3 * B + 1;  // [B]
+  int* s_key = smem_plan + 4 * B + 1;    // [B] columns per item (the sort key)
   for (int b = tid; b < B; b += blockDim.x) {
     int n, start = 0;
     bool bad;
@@ -62,21 +69,23 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
     }
     s_len[b] = bad ? 0 : n;
     s_start[b] = bad ? 0 : start;
+    s_key[b] = work_rows(kind, s_len[b], kr) > 0 ? work_cols(kind, s_len[b], kr) : 0;
   }
   __syncthreads();
-  // Rank of each sequence in the longest-first order (ties keep batch order).
+  // Rank of each sequence in the longest-first order of its items' column
+  // counts (ties keep batch order).
   for (int b = tid; b < B; b += blockDim.x) {
-    const int nb = s_len[b];
+    const int nb = s_key[b];
     int rank = 0;
     for (int o = 0; o < B; ++o) {
-      const int no = s_len[o];
+      const int no = s_key[o];
       rank += (no > nb) || (no == nb && o < b);
     }
     s_order[rank] = b;
   }
   __syncthreads();
   if (tid == 0) s_off[0] = 0;
-  for (int s = tid; s < B; s += blockDim.x) s_off[s + 1] = H * ceil_div(s_len[s_order[s]], rows);
+  for (int s = tid; s < B; s += blockDim.x) s_off[s + 1] = H * ceil_div(work_rows(kind, s_len[s_order[s]], kr), rows);
   __syncthreads();
   // Inclusive scan of s_off[1..B] by warp 0, 32 entries at a time.
   if (tid < 32) {
@@ -110,22 +119,22 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
     }
     const int b = s_order[lo];
     const int local = i - s_off[lo];
-    const int nblk = ceil_div(s_len[b], rows);
+    const int nblk = ceil_div(work_rows(kind, s_len[b], kr), rows);
     items[i] = make_int4(b * H + local / nblk, local % nblk, s_len[b], s_start[b]);
   }
 }
 
-cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, int* ws,
-                        cudaStream_t stream) {
-  const int smem = (4 * B + 1) * static_cast<int>(sizeof(int));
+cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, KeyRange kr,
+                        int* ws, cudaStream_t stream) {
+  const int smem = (5 * B + 1) * static_cast<int>(sizeof(int));
   static PerDeviceOnce attr;
   const cudaError_t e = attr.run([] {
     return cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (4 * kMaxBatch + 1) * static_cast<int>(sizeof(int)));
+                                (5 * kMaxBatch + 1) * static_cast<int>(sizeof(int)));
   });
   if (e != cudaSuccess) return e;
   const int threads = B <= 256 ? 256 : 1024;
-  prep_kernel<<<1, threads, smem, stream>>>(lengths, cu, total, B, H, L, item_rows(kind), ws);
+  prep_kernel<<<1, threads, smem, stream>>>(lengths, cu, total, B, H, L, kind, kr, ws);
   return cudaGetLastError();
 }
 
@@ -135,22 +144,22 @@ cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int
 // slice is cut into `parts` interleaved shares so that the CTAs stay balanced
 // when B*H is small. The final wait keeps the stream order: this grid (and so
 // the call) completes only after the compute kernel before it.
-__global__ void __launch_bounds__(32) fill_kernel(const int* __restrict__ lengths, int B, int H, int L, int d,
-                                                  int rows, int parts, __nv_bfloat16* out0, __nv_bfloat16* out1) {
-  const long long units = static_cast<long long>(B) * H * parts;
-  for (long long u = blockIdx.x; u < units; u += gridDim.x)
-    zero_fill_unit(lengths, H, L, d, rows, parts, u, threadIdx.x, out0, out1);
+__global__ void __launch_bounds__(32) fill_kernel(const int* __restrict__ lengths, int B, FillGeom g, int parts,
+                                                  void* out0, void* out1) {
+  const long long units = static_cast<long long>(B) * g.H * parts;
+  for (long long u = blockIdx.x; u < units; u += gridDim.x) zero_fill_unit(lengths, g, parts, u, threadIdx.x, out0, out1);
   grid_dep_wait();
 }
 
-// The fill overlaps the forward and dK/dV kernels (for dQ the compute kernel
-// zeroes its own uncovered rows in its tail, see bwd.cu).
-cudaError_t launch_fill(const int* lengths, int B, int H, int L, int d, int kind, void* out0, void* out1,
-                        int num_sms, cudaStream_t stream) {
+// The fill overlaps the forward kernel (the backward kernels zero their own
+// uncovered rows, see bwd.cu). elem_bytes is 2 for bf16 outputs and 4 for the
+// fp32 partial sums of a key-range forward.
+cudaError_t launch_fill(const int* lengths, int B, int H, int L, int d, int kind, KeyRange kr, int elem_bytes,
+                        void* out0, void* out1, int num_sms, cudaStream_t stream) {
   const int parts = zero_fill_parts(static_cast<long long>(B) * H, num_sms);
   const int grid = std::max(1, num_sms);
-  return launch_programmatic(fill_kernel, dim3(grid), dim3(32), 0, stream, lengths, B, H, L, d, item_rows(kind),
-                             parts, static_cast<__nv_bfloat16*>(out0), static_cast<__nv_bfloat16*>(out1));
+  const FillGeom g{H, L, kind == kKindDkdv ? kr.count : L, d * elem_bytes / 16, kind, item_rows(kind), kr};
+  return launch_programmatic(fill_kernel, dim3(grid), dim3(32), 0, stream, lengths, B, g, parts, out0, out1);
 }
 
 // Diagnostic: one warp waits, with a bounded wait, on an mbarrier that nothing
@@ -177,16 +186,25 @@ cudaError_t launch_selftest_timeout(int* ws, unsigned long long limit_ns, cudaSt
 // Diagnostic: the sigmoid of scores exactly as the compute kernels evaluate it
 // (sigmoid_score with the kernels' constants for head size D and length n),
 // and its derivative as the backward kernels use it.
+// Each warp takes 32 consecutive scores per step (the sigmoid's branch is
+// warp-uniform, so all 32 lanes stay in the loop; lanes past `count` compute a
+// dummy score and store nothing).
 template <int D>
 __global__ void eval_sigmoid_kernel(const float* __restrict__ s, float* __restrict__ p, float* __restrict__ slope,
                                     int count, int n) {
   const float scale_l2e = Scale<D>::value * kLog2e;
   const float neg_log2n = -__log2f(static_cast<float>(n));
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long base = (blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5)) * 32; base < count;
+       base += warps * 32) {
+    const long long i = base + lane;
     float dp;
-    const float v = sigmoid_score(s[i], scale_l2e, neg_log2n, &dp);
-    p[i] = v;
-    slope[i] = dp;
+    const float v = sigmoid_score(i < count ? s[i] : 0.0f, scale_l2e, neg_log2n, &dp);
+    if (i < count) {
+      p[i] = v;
+      slope[i] = dp;
+    }
   }
 }
 
@@ -197,6 +215,23 @@ cudaError_t launch_eval_sigmoid(const float* s, float* p, float* slope, int coun
     eval_sigmoid_kernel<64><<<grid, 256, 0, stream>>>(s, p, slope, count, n);
   else
     eval_sigmoid_kernel<128><<<grid, 256, 0, stream>>>(s, p, slope, count, n);
+  return cudaGetLastError();
+}
+
+// fp32 -> bf16 (round to nearest even), eight values per thread and step:
+// the last step of a key-sharded call, after its fp32 partial sums were added.
+__global__ void cast_bf16_kernel(const float4* __restrict__ in, uint4* __restrict__ out, long long n8) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = in[2 * i], b = in[2 * i + 1];
+    out[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+}
+
+cudaError_t launch_cast_bf16(const float* in, void* out, long long count, int num_sms, cudaStream_t stream) {
+  const long long n8 = count / 8;
+  const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(8LL * num_sms, (n8 + 255) / 256)));
+  cast_bf16_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(in), static_cast<uint4*>(out), n8);
   return cudaGetLastError();
 }
 
