@@ -12,7 +12,9 @@ Every value it returns is computed in fp64 from the exact values of the inputs
 Source followed: "Better Models, Faster Training: Sigmoid Attention for
 single-cell Foundation Models" -- sec. 2A (SigmoidAttn equation, bias
 b = -log(n)), sec. 2B (sigma' = sigma(1 - sigma), bounded by 0.25; diagonal
-Jacobian), sec. 2C (padding skipped on both sides; dQ and dK/dV gradients).
+Jacobian), sec. 2C (padding skipped on both sides; dQ and dK/dV gradients),
+sec. 4A (the softmax comparison; softmax_forward states softmax attention over
+the valid keys, as the attention-survey page writes it).
 """
 from __future__ import annotations
 
@@ -54,6 +56,8 @@ def _load():
         lib.oracle_bwd.argtypes = [_dp] * 7 + [_ip] + [ctypes.c_int] * 4
         lib.oracle_rows.restype = None
         lib.oracle_rows.argtypes = [_dp] * 4 + [_ip] + [ctypes.c_int] * 5 + [_ip, _ip, ctypes.c_int, _dp]
+        lib.oracle_softmax_fwd.restype = None
+        lib.oracle_softmax_fwd.argtypes = [_dp] * 5 + [_ip] + [ctypes.c_int] * 4
         lib.oracle_tiles.restype = ctypes.c_int
         lib.oracle_tiles.argtypes = [_ip] + [ctypes.c_int] * 4 + [_ip, ctypes.c_int]
         _lib = lib
@@ -101,6 +105,19 @@ def backward(q, k, v, dout, lengths):
     dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
     _load().oracle_bwd(*[_ptr(a, _dp) for a in (q, k, v, dout, dq, dk, dv)], _ptr(lens, _ip), B, H, L, d)
     return dq, dk, dv
+
+
+def softmax_forward(q, k, v, lengths):
+    """The softmax counterpart: (O [B,H,L,d], lse [B,H,L]) over the valid keys,
+    rows i >= n_b zero (see oracle_softmax_fwd_row)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    lens = _i32(lengths)
+    B, H, L, d = q.shape
+    o = np.zeros_like(q)
+    lse = np.zeros((B, H, L), dtype=np.float64)
+    _load().oracle_softmax_fwd(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(o, _dp), _ptr(lse, _dp),
+                               _ptr(lens, _ip), B, H, L, d)
+    return o, lse
 
 
 ROW_KIND = {"o": 0, "dq": 1, "dk": 2, "dv": 3}

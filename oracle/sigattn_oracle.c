@@ -202,3 +202,56 @@ int oracle_tiles(const int* lengths, int B, int H, int L, int block, int* out, i
   }
   return count;
 }
+
+/*
+ * The softmax counterpart, against which the sigmoid kernels are compared on
+ * the same scheduler ("Better Models, Faster Training: Sigmoid Attention for
+ * single-cell Foundation Models", sec. 4A, compares the sigmoid kernel with
+ * softmax attention's FlashAttention-2 at 25% padding; sec. 2A contrasts the
+ * two weightings; the attention-survey page states softmax attention). For one
+ * (b,h) slice and a valid row i < n, over the valid keys j < n only:
+ *
+ *   S_ij  = <Q_i, K_j> / sqrt(d)             (no bias: softmax normalises)
+ *   m_i   = max_{j<n} S_ij
+ *   O_i   = sum_j exp(S_ij - m_i) V_j / sum_j exp(S_ij - m_i)
+ *   lse_i = m_i + ln sum_j exp(S_ij - m_i)
+ *
+ * Rows i >= n are 0 (O and lse), as for the sigmoid path.
+ */
+void oracle_softmax_fwd_row(const double* q, const double* k, const double* v, int n, int d, int i,
+                            double* o_row, double* lse) {
+  for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+  *lse = 0.0;
+  if (i >= n) return;
+  const double scale = 1.0 / sqrt((double)d);
+  const double* qi = q + (size_t)i * d;
+  double m = -INFINITY;
+  for (int j = 0; j < n; ++j) {
+    const double s = scale * dot(qi, k + (size_t)j * d, d);
+    if (s > m) m = s;
+  }
+  double l = 0.0;
+  for (int j = 0; j < n; ++j) {
+    const double p = exp(scale * dot(qi, k + (size_t)j * d, d) - m);
+    l += p;
+    const double* vj = v + (size_t)j * d;
+    for (int c = 0; c < d; ++c) o_row[c] += p * vj[c];
+  }
+  for (int c = 0; c < d; ++c) o_row[c] /= l;
+  *lse = m + log(l);
+}
+
+/* Full softmax forward over [B][H][L][d] (lse: [B][H][L]); parallel over rows. */
+void oracle_softmax_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
+                        const int* lengths, int B, int H, int L, int d) {
+  const long long rows = (long long)B * H * L;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (long long r = 0; r < rows; ++r) {
+    const long long bh = r / L;
+    const int i = (int)(r % L);
+    const int b = (int)(bh / H);
+    const size_t off = (size_t)bh * L * d;
+    oracle_softmax_fwd_row(q + off, k + off, v + off, valid_len(lengths, b, L), d, i, o + off + (size_t)i * d,
+                           lse + (size_t)bh * L + i);
+  }
+}
