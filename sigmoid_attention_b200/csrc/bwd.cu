@@ -224,10 +224,10 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       const float neg_log2n = -__log2f(static_cast<float>(n));  // bias * log2(e)
       for (int j = 0; j < nb; ++j) {
         // ---- S -> sigma'(x) = P (1 - P) kept in registers for dS, and (dK/dV)
-        // bf16 P for dV, stored chunk by chunk as it is computed (the P region
-        // is free once the previous block's dV products have read it). Padded
-        // columns get P = sigma' = 0.
+        // bf16 P for dV, written once the previous block's dV products have
+        // read the P region. Padded columns get P = sigma' = 0.
         float sp[CPW][32];
+        uint32_t pk[KV ? CPW : 1][16];
         {
           uint32_t sv[CPW][32];
           if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, ws, 221))) break;
@@ -240,61 +240,52 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.xs_read);
-          if (KV) {
-            if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
-            tc_fence_after();
-          }
           const int valid = ncols - (j * C::BN + g * CPW * 32);  // columns < valid are real tokens
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
-            uint32_t pk[16];
             mask_scores(sv[c], valid - 32 * c, row_ok);
             sigmoid32<true>(sv[c], scale_l2e, neg_log2n, sp[c]);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              pk[e] = pack_bf16x2(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1]));
             if (KV) {
-              tmem_st16(tmem + lane_off + C::TM_P + (g * CPW + c) * 16, pk);
-              tmem_st_wait();
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&bar.p_full[g * CPW + c]);
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                pk[KV ? c : 0][e] = pack_bf16x2(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1]));
             }
           }
         }
-        // ---- dP -> dS = dP P (1 - P), bf16 dS for dQ / dK. The dK/dV kernel
-        // (fewer registers per thread) copies dP out one chunk at a time.
-        constexpr bool kDpAtOnce = !KV;
-        uint32_t dp[kDpAtOnce ? CPW : 1][32];
+        if (KV) {
+          if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < CPW; ++c) {
+            tmem_st16(tmem + lane_off + C::TM_P + (g * CPW + c) * 16, pk[KV ? c : 0]);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.p_full[g * CPW + c]);
+          }
+        }
+        // ---- dP -> dS = dP P (1 - P), bf16 dS for dQ / dK: dP is copied out
+        // whole, so its region is released at once.
+        uint32_t dp[CPW][32];
         const uint32_t tXDP = xb ? tXDP1 : tXDP0;
         uint64_t* xdp_read = &bar.xdp_read[xb];
         if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, ws, 222))) break;
         dp_ph[xb] ^= 1;
         if (++xb == static_cast<uint32_t>(C::NXDP)) xb = 0;
         tc_fence_after();
-        if (kDpAtOnce) {
 #pragma unroll
-          for (int c = 0; c < CPW; ++c) tmem_ld32_async(tXDP + 32 * c, dp[kDpAtOnce ? c : 0]);
+        for (int c = 0; c < CPW; ++c) tmem_ld32_async(tXDP + 32 * c, dp[c]);
 #pragma unroll
-          for (int c = 0; c < CPW; ++c) tmem_ld_wait32(dp[kDpAtOnce ? c : 0]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(xdp_read);
-        }
+        for (int c = 0; c < CPW; ++c) tmem_ld_wait32(dp[c]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xdp_read);
         if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, ws, 224))) break;
         free_ph ^= 1;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < CPW; ++c) {
-          uint32_t(&dpc)[32] = dp[kDpAtOnce ? c : 0];
-          if (!kDpAtOnce) {
-            tmem_ld32(tXDP + 32 * c, dpc);
-            if (c + 1 == CPW) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(xdp_read);
-            }
-          }
+          const uint32_t(&dpc)[32] = dp[c];
           uint32_t dk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
