@@ -322,6 +322,47 @@ def side_workloads(names, dev, steps: int, warmup: int) -> dict:
     return out
 
 
+def softmax_comparison(name: str, dev, steps: int = 10, warmup: int = 3) -> dict:
+    """Forward TFLOPS of the sigmoid kernel and of its softmax counterpart
+    (same plan, scheduler, loads and MMAs; softmax over the valid keys) on
+    one workload, device-timed the same way (L2 flushed between steps): the
+    comparison of "Better Models, Faster Training" sec. 4A, at its 25%
+    padding when run on pad_sweep_p25."""
+    import torch
+
+    import sigmoid_attention_b200 as sa
+    from sigmoid_attention_b200 import workloads
+
+    w = workloads.WORKLOADS[name]
+    q, k, v, _, lengths = workloads.workload_inputs(w)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    lens = lengths.to(dev)
+    o = torch.empty_like(qd)
+    ws = sa.make_workspace(w.B, w.H, w.L, w.d, dev)
+    stream = torch.cuda.current_stream(dev)
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    out = {"workload": name, "steps": steps}
+    for key, call in (("sigmoid", lambda: sa.sigattn_fwd(qd, kd, vd, o, lens, ws, stream)),
+                      ("softmax", lambda: sa.sigattn_softmax_fwd(qd, kd, vd, o, lens, ws, stream))):
+        for _ in range(warmup):
+            call()
+            flush_buf.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+        torch.cuda.synchronize(dev)
+        for i in range(steps):
+            ev[2 * i].record(stream)
+            call()
+            ev[2 * i + 1].record(stream)
+            flush_buf.zero_()
+        torch.cuda.synchronize(dev)
+        _check_status(sa, ws, stream)
+        ms = float(np.mean([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)]))
+        out[f"{key}_fwd_ms"] = ms
+        out[f"{key}_fwd_tflops"] = w.fwd_flops() / (ms / 1e3) / 1e12
+    out["sigmoid_over_softmax"] = out["sigmoid_fwd_tflops"] / out["softmax_fwd_tflops"]
+    return out
+
+
 def unfused_torch(w, q, k, v, dout, lengths, dev, steps: int = 5, warmup: int = 3) -> dict:
     """The comparison of "Better Models, Faster Training" sec. 4A: sigmoid
     attention written as plain PyTorch operations (bf16 matmuls, an explicit
@@ -612,6 +653,7 @@ def run_gpu(args, w):
         # (device-timed), and the unfused PyTorch comparison on this workload.
         side = [n_ for n_ in ("pad_sweep_p00", "pad_sweep_p75", "scrna_ragged", "long_8k") if n_ != w.name]
         line["other_workloads"] = side_workloads(side, dev, steps=10, warmup=3)
+        line["softmax_counterpart"] = softmax_comparison("pad_sweep_p25", dev)
         if w.name in ("pad_sweep_p00", "pad_sweep_p75"):
             mine = {"value": value, "fwd_tflops": fwd_tflops, "bwd_tflops": bwd_tflops}
             other = line["other_workloads"].get("pad_sweep_p75" if w.name == "pad_sweep_p00" else "pad_sweep_p00")

@@ -148,6 +148,20 @@ SIGATTN_API int sigattn_bwd_dkdv_range(const void* q, const void* k, const void*
                                        void* dv, const int32_t* lengths, int B, int H, int Lmax, int d, int key_begin,
                                        int key_count, void* workspace, size_t workspace_bytes, void* stream);
 
+/* The softmax counterpart of sigattn_fwd, for comparisons on equal terms
+ * (Better Models, Faster Training, sec. 4A compares the sigmoid kernel with
+ * softmax attention's FlashAttention-2 on padded batches): the same plan,
+ * scheduler, data movement and MMAs, with the sigmoid replaced by a softmax
+ * over each sequence's valid keys,
+ *     O_i = sum_{j<n} exp(S_ij) V_j / sum_{j<n} exp(S_ij),  S = Q K^T / sqrt(d),
+ * computed online (running row maximum, lazily rescaled O and row sums).
+ * Forward only, d = 64 only (SIGATTN_ERR_UNSUPPORTED otherwise), padded
+ * layout; arguments, outputs (rows >= n_b zero) and workspace as sigattn_fwd.
+ * No log-sum-exp is returned. */
+SIGATTN_API int sigattn_softmax_fwd(const void* q, const void* k, const void* v, void* o, const int32_t* lengths,
+                                    int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
 /* Round `count` fp32 values to bf16 (nearest even), x -> y, both device
  * pointers, 16-byte aligned; count a multiple of 8. The last step after the
  * fp32 partial sums of key ranges were added (e.g. by an all-reduce). */

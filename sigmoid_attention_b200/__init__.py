@@ -24,6 +24,7 @@ __all__ = [
     "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "sigattn_eval_sigmoid", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
     "sigattn_fwd_varlen", "sigattn_bwd_dq_varlen", "sigattn_bwd_dkdv_varlen",
     "sigattn_fwd_partial", "sigattn_bwd_dq_partial", "sigattn_bwd_dkdv_range", "sigattn_cast_bf16",
+    "sigattn_softmax_fwd",
     "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
     "SigmoidAttentionVarlenFunction", "sigmoid_attention_varlen",
 ]
@@ -94,6 +95,8 @@ def library():
         lib.sigattn_bwd_dq_partial.argtypes = [_vp] * 6 + [_i] * 6 + [_vp, _sz, _vp]
         lib.sigattn_bwd_dkdv_range.restype = _i
         lib.sigattn_bwd_dkdv_range.argtypes = [_vp] * 7 + [_i] * 6 + [_vp, _sz, _vp]
+        lib.sigattn_softmax_fwd.restype = _i
+        lib.sigattn_softmax_fwd.argtypes = [_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp]
         lib.sigattn_cast_bf16.restype = _i
         lib.sigattn_cast_bf16.argtypes = [_vp, _vp, ctypes.c_longlong, _vp]
         lib.sigattn_eval_sigmoid.restype = _i
@@ -157,6 +160,14 @@ def make_workspace(B: int, H: int, Lmax: int, d: int, device=None) -> torch.Tens
 def sigattn_fwd(q, k, v, o, lengths, workspace, stream=None) -> None:
     B, H, L, d = _dims(q)
     _check("sigattn_fwd", library().sigattn_fwd(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lengths, "lengths", torch.int32),
+        B, H, L, d, _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_softmax_fwd(q, k, v, o, lengths, workspace, stream=None) -> None:
+    """The softmax counterpart of sigattn_fwd (d = 64, forward only)."""
+    B, H, L, d = _dims(q)
+    _check("sigattn_softmax_fwd", library().sigattn_softmax_fwd(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lengths, "lengths", torch.int32),
         B, H, L, d, _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
 

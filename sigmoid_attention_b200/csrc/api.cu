@@ -24,6 +24,8 @@ cudaError_t launch_cast_bf16(const float* in, void* out, long long count, int nu
 cudaError_t launch_fwd(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, void* o, int* ws, int B, int H, int L, KeyRange kr, int num_sms,
                        cudaStream_t stream);
+cudaError_t launch_softmax_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
+                               int B, int H, int L, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_dq(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tdo,
                           const CUtensorMap& tk, const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L,
                           KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream);
@@ -339,6 +341,25 @@ int sigattn_bwd_dkdv_range(const void* q, const void* k, const void* v, const vo
                            void* workspace, size_t workspace_bytes, void* stream) {
   return dkdv_padded(q, k, v, dout, dk, dv, lengths, B, H, Lmax, d, KeyRange{key_begin, key_count}, workspace,
                      workspace_bytes, stream);
+}
+
+int sigattn_softmax_fwd(const void* q, const void* k, const void* v, void* o, const int32_t* lengths, int B, int H,
+                        int Lmax, int d, void* workspace, size_t workspace_bytes, void* stream) {
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (d != 64) return SIGATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SIGATTN_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) || !make_map(&tv, v, B * H, Lmax, d))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws = static_cast<int*>(workspace);
+  const KeyRange all{0, Lmax};
+  st = cuda_status(launch_prep(lengths, nullptr, 0, B, H, Lmax, SIGATTN_KIND_FWD, all, ws, s));
+  if (st == SIGATTN_OK) st = cuda_status(launch_softmax_fwd(tq, tk, tv, o, ws, B, H, Lmax, info.num_sms, s));
+  if (st != SIGATTN_OK) return st;
+  return cuda_status(launch_fill(lengths, B, H, Lmax, d, SIGATTN_KIND_FWD, all, 2, o, nullptr, info.num_sms, s));
 }
 
 int sigattn_cast_bf16(const float* x, void* y, long long count, void* stream) {

@@ -76,6 +76,8 @@ struct FwdBarriers {
   uint64_t s_read[2];    // SEP_P: the epilogue copied tile t's S out of TMEM (S region free)
   uint64_t pv_done[2];   // SEP_P: tile t's PV products of a block completed (P region free)
   uint64_t drain[2];
+  uint64_t xmax[4][2];  // softmax: the four warps of a lane quadrant wrote their row maxima (by pass parity)
+  uint64_t xsum[4];     // softmax: ... their partial row sums (end of an item)
   ItemRing ring;
   uint32_t tmem_base;
   int abort;
@@ -83,14 +85,24 @@ struct FwdBarriers {
 
 // F32OUT: the output is the fp32 partial sum over the call's key range (no
 // rounding to bf16), for key-range calls whose partial outputs are summed.
-template <int D, bool PACKED, bool F32OUT>
+// SOFTMAX (D = 64, padded layout, whole sequences): softmax attention over the
+// valid keys instead of the sigmoid, on the same scheduler, producer and MMA
+// issuers (the counterpart that the comparison of Better Models sec. 4A
+// needs): only the epilogue differs (online row maximum exchanged between the
+// four warps that share a row, lazily rescaled O and row sums, O / l at the end).
+template <int D, bool PACKED, bool F32OUT, bool SOFTMAX>
 __global__ void __launch_bounds__((16 + 3) * 32, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, void* __restrict__ out, int* __restrict__ ws, int H, int L,
                KeyRange kr) {
   using C = FwdCfg<D>;
+  static_assert(!SOFTMAX || (C::SEP_P && !PACKED && !F32OUT), "softmax: d = 64, padded layout, bf16 output");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ FwdBarriers<C::KST, C::VST> bar;
+  // Softmax only: the row maxima of a pass (two buffers, by pass parity) and
+  // the row sums at the end of an item, per tile, column chunk and row.
+  __shared__ float soft_max[SOFTMAX ? 2 * 4 * 128 : 1];
+  __shared__ float soft_sum[SOFTMAX ? 2 * 4 * 128 : 1];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sK = smem + C::OFF_K;
@@ -122,6 +134,11 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
     mbar_init(&bar.epi_done[1], 8);
     mbar_init(&bar.drain[0], 1);
     mbar_init(&bar.drain[1], 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&bar.xmax[q][0], 4);
+      mbar_init(&bar.xmax[q][1], 4);
+      mbar_init(&bar.xsum[q], 4);
+    }
     ring_init(bar.ring, 2 + C::EPI_WARPS);  // both issuers and every epilogue warp read each item
     bar.abort = 0;
     fence_mbar_init();
@@ -336,6 +353,148 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       mma_commit(&bar.drain[t]);
       mbar_wait(&bar.drain[t], 0, &never, ws, 119);
     }
+  } else if constexpr (SOFTMAX) {
+    // -------------------------------------------- softmax epilogue (D = 64)
+    // Warp w covers lane quadrant qd = w & 3 and key columns [32c, 32c + 32),
+    // c = w >> 2, as in the sigmoid epilogue below. Per pass (tile t, key
+    // block j) each warp takes its chunk's row maximum; the four warps of a
+    // quadrant exchange them through shared memory (an mbarrier per quadrant
+    // and buffer parity, waited with the same bound as every other hand-off),
+    // so all four hold the same block maximum and the same running maximum m.
+    // m only moves when the block maximum exceeds it by more than kTau
+    // (log2 units), and then O and the partial row sums l are rescaled by
+    // 2^(m_old - m_new) (warps c = 0, 1 rescale the tile's 64 O columns, before
+    // they signal the first P half, which the issuer waits for before the
+    // block's first PV product). P = 2^(y - m) with y = s * scale * log2(e).
+    // At the end of an item the four partial row sums are added through
+    // shared memory and O is divided by them.
+    constexpr float kTau = 8.0f;
+    const int c = warp >> 2, qd = warp & 3;
+    const int r = (qd << 5) + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(qd << 5) << 16;
+    const int ot = c >> 1, oc = c & 1;
+    constexpr float scale_l2e = Scale<D>::value * kLog2e;
+    uint32_t sph[2] = {0, 0}, oph[2] = {0, 0}, pvph[2] = {0, 0};
+    bool pv_pending[2] = {false, false};
+    uint32_t pass = 0, sum_ph = 0;
+    bool ok = true;
+    uint32_t ist = 0, iph = 0;
+    while (ok) {
+      Item item;
+      if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 120))) break;
+      __syncwarp();
+      ring_release(bar.ring, ist, iph, lane == 0);
+      if (item.n < 0) break;
+      const int n = item.n;
+      const int row_base = item.blk * (C::BM * C::NQ);
+      const int ntiles = (row_base + C::BM < n) ? 2 : 1;
+      const int nkb = ceil_div(n, C::BN);
+      float m[2] = {0.f, 0.f}, l[2] = {0.f, 0.f};
+      for (int j = 0; ok && j < nkb; ++j) {
+        const int valid = n - (j * C::BN + 32 * c);  // columns < valid are real keys
+        for (int t = 0; t < ntiles; ++t) {
+          if (!(ok = mbar_wait(&bar.s_full[t], sph[t], abort_flag, ws, 121))) break;
+          sph[t] ^= 1;
+          tc_fence_after();
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + C::TM_S + t * 128 + 32 * c, a);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.s_read[t]);
+          // y in log2 units; keys past n get -inf, rows past n (discarded) 0
+          const bool row_ok = row_base + t * C::BM + r < n;
+          float cm = -INFINITY;  // a[e] becomes y, in place
+          if (valid >= 32 && row_ok) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float y = __uint_as_float(a[e]) * scale_l2e;
+              a[e] = __float_as_uint(y);
+              cm = fmaxf(cm, y);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float y = !row_ok ? 0.0f : (e < valid ? __uint_as_float(a[e]) * scale_l2e : -INFINITY);
+              a[e] = __float_as_uint(y);
+              cm = fmaxf(cm, y);
+            }
+          }
+          float* mx = soft_max + (pass & 1) * 512;
+          mx[c * 128 + r] = cm;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.xmax[qd][pass & 1]);
+          if (!(ok = mbar_wait(&bar.xmax[qd][pass & 1], (pass >> 1) & 1, abort_flag, ws, 125))) break;
+          const float bm = fmaxf(fmaxf(mx[r], mx[128 + r]), fmaxf(mx[256 + r], mx[384 + r]));
+          ++pass;
+          // O and the P region are free once the tile's previous PV products completed.
+          if (pv_pending[t]) {
+            if (!(ok = mbar_wait(&bar.pv_done[t], pvph[t], abort_flag, ws, 124))) break;
+            pvph[t] ^= 1;
+          }
+          pv_pending[t] = true;
+          tc_fence_after();
+          if (j == 0) {
+            m[t] = bm;  // the block's first PV product overwrites O
+            l[t] = 0.f;
+          } else if (__any_sync(0xffffffffu, bm > m[t] + kTau)) {
+            const float mn = fmaxf(m[t], bm);
+            const float alpha = ex2_approx(m[t] - mn);
+            m[t] = mn;
+            l[t] *= alpha;
+            if (c < 2) {
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t to = tmem + lane_off + C::TM_O + t * D + 32 * c + 16 * hf;
+                uint32_t o[16];
+                tmem_ld16(to, o);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                tmem_st16(to, o);
+              }
+            }
+          }
+          uint32_t pk[16];
+          float ls = 0.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(__uint_as_float(a[2 * e]) - m[t]);
+            const float p1 = ex2_approx(__uint_as_float(a[2 * e + 1]) - m[t]);
+            ls += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          l[t] += ls;
+          tmem_st16(tmem + lane_off + C::TM_P + t * 64 + 16 * c, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.p_full[2 * t + (c >> 1)]);
+        }
+      }
+      if (!ok) break;
+      // Row sums: the four partials of each row, added through shared memory.
+      for (int t = 0; t < ntiles; ++t) soft_sum[t * 512 + c * 128 + r] = l[t];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.xsum[qd]);
+      if (!(ok = mbar_wait(&bar.xsum[qd], sum_ph, abort_flag, ws, 126))) break;
+      sum_ph ^= 1;
+      const int row = row_base + ot * C::BM + r;
+      const size_t orow = rm.offset(item, 0, row, D) + 32 * oc;
+      if (ot >= ntiles) {  // tile fully padded: its rows of O are zero
+        if (rm.writes(row, n)) store_zero_out32<false>(out, orow);
+        continue;
+      }
+      const float* ps = soft_sum + ot * 512;
+      const float inv_l = 1.0f / (ps[r] + ps[128 + r] + ps[256 + r] + ps[384 + r]);
+      if (!(ok = mbar_wait(&bar.o_full[ot], oph[ot], abort_flag, ws, 122))) break;
+      oph[ot] ^= 1;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + C::TM_O + ot * D + 32 * oc, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.o_empty[ot]);
+      if (rm.writes(row, n)) store_out32<false>(out, orow, v, inv_l, row >= n);
+    }
   } else if constexpr (C::SEP_P) {
     // ------------------------------------------------- epilogue (D = 64, SEP_P)
     // All 16 warps take each tile's sigmoid pass in turn (tile 0, then tile 1,
@@ -509,20 +668,26 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
   }
 }
 
-template <int D, bool PACKED, bool F32OUT>
+template <int D, bool PACKED, bool F32OUT, bool SOFTMAX = false>
 cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
                             int B, int H, int L, KeyRange kr, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D>;
   static PerDeviceOnce attr;
   const cudaError_t e = attr.run([] {
-    return cudaFuncSetAttribute(fwd_kernel<D, PACKED, F32OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(fwd_kernel<D, PACKED, F32OUT, SOFTMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 C::SMEM_ALLOC);
   });
   if (e != cudaSuccess) return e;
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kFwdItemRows);
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
-  return launch_programmatic(fwd_kernel<D, PACKED, F32OUT>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream, tq,
-                             tk, tv, o, ws, H, L, kr);
+  return launch_programmatic(fwd_kernel<D, PACKED, F32OUT, SOFTMAX>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC,
+                             stream, tq, tk, tv, o, ws, H, L, kr);
+}
+
+// The softmax counterpart (d = 64, padded layout).
+cudaError_t launch_softmax_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
+                               int B, int H, int L, int num_sms, cudaStream_t stream) {
+  return launch_fwd_impl<64, false, false, true>(tq, tk, tv, o, ws, B, H, L, KeyRange{0, L}, num_sms, stream);
 }
 
 // L is Lmax for the padded layout and the longest sequence for the packed one.
