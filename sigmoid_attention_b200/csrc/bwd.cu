@@ -33,13 +33,15 @@
 // BN is 128, except for dK/dV at D = 128, where the two D-wide accumulators
 // leave room in the 512 TMEM columns only for 64-column S and dP regions:
 //   XS [0,BN) XdP [BN,2BN) P [2BN,2.5BN) dS [2.5BN,3BN) A1 [3BN,3BN+D) A2 after.
-// Warps: 0-7 epilogue (warps 4g..4g+3 take columns [g BN/2, (g+1) BN/2) of
-// each block), 8 TMA producer (also claims the work items and passes them on
-// through the shared-memory item ring; for dQ at D = 64 over padded inputs it
-// also writes the zeros of the rows no item covers, with bulk copies from
-// shared memory while the compute runs), 9 S issuer (owns TMEM), 10 dP issuer,
-// 11 A1 issuer, 12 A2 issuer (dK/dV only). PACKED selects the input layout, as
-// in the forward kernel.
+// Warps: 0 .. E-1 epilogue, E = 4 G with G column groups (warps 4g..4g+3 take
+// columns [g BN/G, (g+1) BN/G) of each block, in chunks of CW columns; G = 2,
+// CW = 32), then the TMA
+// producer (also claims the work items and passes them on through the
+// shared-memory item ring; for dQ at D = 64 over padded inputs it also writes
+// the zeros of the rows no item covers, with bulk copies from shared memory
+// while the compute runs), the S issuer (owns TMEM), the dP issuer, the A1
+// issuer and (dK/dV) the A2 issuer; idle warps round the CTA up to whole
+// warpgroups. PACKED selects the input layout, as in the forward kernel.
 #include "common.cuh"
 
 namespace sigattn {
@@ -48,8 +50,15 @@ template <int D, bool KV>
 struct BwdCfg {
   static constexpr int BM = kBwdItemRows;   // 128 rows per item
   static constexpr int BN = bwd_col_block(KV, D);
-  static constexpr int NCH = BN / 32;       // 32-column chunks per block
-  static constexpr int CPW = NCH / 2;       // chunks per epilogue warp
+  // Epilogue column groups (warps per lane quadrant) and chunk width: 8
+  // epilogue warps on 32-column chunks. (16 warps on 16-column chunks for
+  // dK/dV at D = 128, at 88 registers each, measured slower: 0.918 -> 0.984 ms
+  // on the dense d = 128 workload.)
+  static constexpr int GROUPS = 2;
+  static constexpr int CW = 32;
+  static constexpr int NCH = BN / CW;       // chunks per block
+  static constexpr int CPW = NCH / GROUPS;  // chunks per epilogue warp
+  static_assert(CPW >= 1 && NCH <= 4, "chunking");
   static constexpr int BOX_R = 128 * 64 * 2;   // [128 rows][64 cols] bf16
   static constexpr int BOX_C = BN * 64 * 2;    // [BN rows][64 cols] bf16
   static constexpr int TILE_R = 128 * D * 2;
@@ -80,18 +89,23 @@ struct BwdCfg {
   static constexpr int TM_XDP1 = TM_A1 + (KV ? 2 : 1) * D;
   static constexpr int NXDP = (TM_XDP1 + BN <= TMEM_COLS) ? 2 : 1;
   static_assert(SMEM_ALLOC <= 227 * 1024 - 1024, "shared memory budget");
-  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_WARPS = 4 * GROUPS;
   static constexpr int ISSUERS = KV ? 4 : 3;
-  // Four warpgroups: two of epilogue warps, then the producer, the issuers and
-  // idle warps. The single-thread roles give registers to the epilogue
-  // (setmaxnreg): launched at 128 per thread, 8 warps x 184 + 8 x 64 fit the
-  // 65536 registers of the SM.
-  static constexpr int THREADS = 16 * 32;
-  static constexpr int EPI_REGS = 184;
-  static constexpr int OTHER_REGS = 64;
-  static_assert(EPI_WARPS + 1 + ISSUERS <= 16, "warp roles");
-  static_assert((EPI_WARPS * EPI_REGS + (16 - EPI_WARPS) * OTHER_REGS) * 32 <= 65536, "register split");
-  static_assert(THREADS * 128 <= 65536, "launch registers");
+  // Whole warpgroups: the epilogue's, then one or two holding the producer,
+  // the issuers and idle warps. The single-thread roles give registers to the
+  // epilogue (setmaxnreg). The launch gives every thread LAUNCH_REGS; the
+  // split must not exceed that total (the launcher also checks it against
+  // the count the compiler actually allocated).
+  static constexpr int WARPS = (EPI_WARPS + 1 + ISSUERS + 3) / 4 * 4 < 16 ? 16 : (EPI_WARPS + 1 + ISSUERS + 3) / 4 * 4;
+  static constexpr int THREADS = WARPS * 32;
+  static constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
+  static constexpr int OTHER_REGS = WARPS > 16 ? 56 : 64;
+  static constexpr int EPI_REGS =
+      ((LAUNCH_REGS * WARPS - OTHER_REGS * (WARPS - EPI_WARPS)) / EPI_WARPS) / 8 * 8 > 184
+          ? 184
+          : ((LAUNCH_REGS * WARPS - OTHER_REGS * (WARPS - EPI_WARPS)) / EPI_WARPS) / 8 * 8;
+  static_assert(EPI_REGS * EPI_WARPS + OTHER_REGS * (WARPS - EPI_WARPS) <= LAUNCH_REGS * WARPS, "register split");
+  static_assert(EPI_REGS >= LAUNCH_REGS && OTHER_REGS <= LAUNCH_REGS, "setmaxnreg directions");
 };
 
 template <int ST1, int ST2>
@@ -198,13 +212,13 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   if (warp < C::EPI_WARPS) {
     // ------------------------------------------------------------- epilogue
     setmaxnreg_inc<C::EPI_REGS>();
-    constexpr int CPW = C::CPW;
+    constexpr int CPW = C::CPW, CW = C::CW, G = C::GROUPS;
     const int g = warp >> 2;                      // chunks g*CPW .. g*CPW + CPW - 1
     const int r = ((warp & 3) << 5) + lane;       // row within the item = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
-    const uint32_t tXS = tmem + lane_off + C::TM_XS + g * CPW * 32;
-    const uint32_t tXDP0 = tmem + lane_off + C::TM_XDP + g * CPW * 32;
-    const uint32_t tXDP1 = tmem + lane_off + C::TM_XDP1 + g * CPW * 32;
+    const uint32_t tXS = tmem + lane_off + C::TM_XS + g * CPW * CW;
+    const uint32_t tXDP0 = tmem + lane_off + C::TM_XDP + g * CPW * CW;
+    const uint32_t tXDP1 = tmem + lane_off + C::TM_XDP1 + g * CPW * CW;
     constexpr float scale = Scale<D>::value;
     constexpr float scale_l2e = scale * kLog2e;
     uint32_t s_ph = 0, free_ph = 0, aph = 0, xb = 0;
@@ -226,28 +240,28 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         // ---- S -> sigma'(x) = P (1 - P) kept in registers for dS, and (dK/dV)
         // bf16 P for dV, written once the previous block's dV products have
         // read the P region. Padded columns get P = sigma' = 0.
-        float sp[CPW][32];
-        uint32_t pk[KV ? CPW : 1][16];
+        float sp[CPW][CW];
+        uint32_t pk[KV ? CPW : 1][CW / 2];
         {
-          uint32_t sv[CPW][32];
+          uint32_t sv[CPW][CW];
           if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, ws, 221))) break;
           s_ph ^= 1;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < CPW; ++c) tmem_ld32_async(tXS + 32 * c, sv[c]);
+          for (int c = 0; c < CPW; ++c) tmem_ld_async(tXS + CW * c, sv[c]);
 #pragma unroll
-          for (int c = 0; c < CPW; ++c) tmem_ld_wait32(sv[c]);
+          for (int c = 0; c < CPW; ++c) tmem_ld_wait(sv[c]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.xs_read);
-          const int valid = ncols - (j * C::BN + g * CPW * 32);  // columns < valid are real tokens
+          const int valid = ncols - (j * C::BN + g * CPW * CW);  // columns < valid are real tokens
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
-            mask_scores(sv[c], valid - 32 * c, row_ok);
-            sigmoid32<true>(sv[c], scale_l2e, neg_log2n, sp[c]);
+            mask_scores(sv[c], valid - CW * c, row_ok);
+            sigmoid_n<true>(sv[c], scale_l2e, neg_log2n, sp[c]);
             if (KV) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e)
+              for (int e = 0; e < CW / 2; ++e)
                 pk[KV ? c : 0][e] = pack_bf16x2(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1]));
             }
           }
@@ -257,7 +271,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
-            tmem_st16(tmem + lane_off + C::TM_P + (g * CPW + c) * 16, pk[KV ? c : 0]);
+            tmem_st(tmem + lane_off + C::TM_P + (g * CPW + c) * (CW / 2), pk[KV ? c : 0]);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -266,7 +280,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         }
         // ---- dP -> dS = dP P (1 - P), bf16 dS for dQ / dK: dP is copied out
         // whole, so its region is released at once.
-        uint32_t dp[CPW][32];
+        uint32_t dp[CPW][CW];
         const uint32_t tXDP = xb ? tXDP1 : tXDP0;
         uint64_t* xdp_read = &bar.xdp_read[xb];
         if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, ws, 222))) break;
@@ -274,9 +288,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         if (++xb == static_cast<uint32_t>(C::NXDP)) xb = 0;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < CPW; ++c) tmem_ld32_async(tXDP + 32 * c, dp[c]);
+        for (int c = 0; c < CPW; ++c) tmem_ld_async(tXDP + CW * c, dp[c]);
 #pragma unroll
-        for (int c = 0; c < CPW; ++c) tmem_ld_wait32(dp[c]);
+        for (int c = 0; c < CPW; ++c) tmem_ld_wait(dp[c]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(xdp_read);
@@ -285,13 +299,13 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < CPW; ++c) {
-          const uint32_t(&dpc)[32] = dp[c];
-          uint32_t dk[16];
+          const uint32_t(&dpc)[CW] = dp[c];
+          uint32_t dk[CW / 2];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
+          for (int e = 0; e < CW / 2; ++e)
             dk[e] = pack_bf16x2(__uint_as_float(dpc[2 * e]) * sp[c][2 * e],
                                 __uint_as_float(dpc[2 * e + 1]) * sp[c][2 * e + 1]);
-          tmem_st16(tmem + lane_off + C::TM_DS + (g * CPW + c) * 16, dk);
+          tmem_st(tmem + lane_off + C::TM_DS + (g * CPW + c) * (CW / 2), dk);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
@@ -307,16 +321,17 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       const bool valid_row = row < (KV ? range_keys(n, kr) : n);
       const size_t row_off = rm.offset(item, PACKED ? item.bh % H : 0, row, D);
       // 32-column chunks of the accumulators: A1 (-> out1, times scale), then
-      // A2 (-> out2) for dK/dV; each half of the warps takes every other
-      // chunk. Each chunk is copied out and packed to bf16 at once, so the
+      // A2 (-> out2) for dK/dV; column group g takes chunks g, g + G, ...
+      // Each chunk is copied out and packed to bf16 at once, so the
       // accumulators are released before the (slower) global stores.
       constexpr int kChunks = (KV ? 2 : 1) * (D / 32);
-      constexpr int kPer = kChunks / 2;
+      constexpr int kPer = kChunks / G;
+      static_assert(kPer * G == kChunks, "accumulator chunks");
       // bf16 pairs, or (F32OUT) the fp32 values themselves
       uint32_t packed[kPer][F32OUT ? 32 : 16];
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
-        const int c = g + 2 * i;
+        const int c = g + G * i;
         const bool second = c >= D / 32;
         const int col = (second ? c - D / 32 : c) * 32;
         const float mul = (second ? 1.0f : scale) * (valid_row ? 1.0f : 0.0f);
@@ -337,7 +352,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       if (in_range) {
 #pragma unroll
         for (int i = 0; i < kPer; ++i) {
-          const int c = g + 2 * i;
+          const int c = g + G * i;
           const bool second = c >= D / 32;
           const int col = (second ? c - D / 32 : c) * 32;
           void* out = second ? out2 : out1;
@@ -530,12 +545,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
                 aph ^= 1;
               }
               tc_fence_after();
-              // K = the chunk's 32 columns: two K=16 steps; the chunk's bf16
-              // values sit in 16 TMEM columns (two per column).
+              // K = the chunk's CW columns in K=16 steps; the chunk's bf16
+              // values sit in CW/2 TMEM columns (two per column).
   #pragma unroll
-              for (int kk = 0; kk < 2; ++kk)
-                mma_ts(tm_acc, tm_a + q * 16 + kk * 8, b0 + ((q * 32 * 128 + kk * 2048) >> 4), idesc_acc,
-                       (first && kk == 0) ? 0u : 1u);
+              for (int kk = 0; kk < C::CW / 16; ++kk)
+                mma_ts(tm_acc, tm_a + q * (C::CW / 2) + kk * 8, b0 + ((q * C::CW * 128 + kk * 2048) >> 4),
+                       idesc_acc, (first && kk == 0) ? 0u : 1u);
             }
             if (!ok) break;
             mma_commit(freed);
@@ -584,8 +599,18 @@ cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const 
   using C = BwdCfg<D, KV>;
   static PerDeviceOnce attr;
   const cudaError_t e = attr.run([] {
-    return cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED, F32OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                C::SMEM_ALLOC);
+    cudaError_t r = cudaFuncSetAttribute(bwd_kernel<D, KV, PACKED, F32OUT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+    if (r != cudaSuccess) return r;
+    // The setmaxnreg split draws on the registers the CTA is launched with:
+    // refuse to launch if the compiler allocated fewer than the split needs
+    // (the epilogue's increase would otherwise wait for ever).
+    cudaFuncAttributes fa;
+    r = cudaFuncGetAttributes(&fa, bwd_kernel<D, KV, PACKED, F32OUT>);
+    if (r != cudaSuccess) return r;
+    const long long need = (static_cast<long long>(C::EPI_REGS) * C::EPI_WARPS +
+                            static_cast<long long>(C::OTHER_REGS) * (C::WARPS - C::EPI_WARPS)) * 32;
+    return static_cast<long long>(fa.numRegs) * C::THREADS >= need ? cudaSuccess : cudaErrorLaunchOutOfResources;
   });
   if (e != cudaSuccess) return e;
   const long long max_items = static_cast<long long>(B) * H * ceil_div(L, kBwdItemRows);

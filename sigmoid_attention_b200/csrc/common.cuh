@@ -264,19 +264,20 @@ constexpr float kTailC = 0.0625f;
 // about a thousand: the bias -ln n puts the typical weight near 1/n), the
 // short tail form serves; otherwise the general form. Pairs of columns
 // (2e, 2e + 1) go through the packed fp32x2 FMAs.
-template <bool SLOPE>
-__device__ __forceinline__ void sigmoid32(uint32_t (&a)[32], float scale_l2e, float neg_log2n, float* slope) {
+template <bool SLOPE, int N>
+__device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, float neg_log2n, float* slope) {
+  static_assert(N == 16 || N == 32, "16 or 32 scores per thread");
   const uint64_t c1 = f2_splat(scale_l2e), c0 = f2_splat(neg_log2n - kTailY);
-  uint64_t z[16];  // z = y - kTailY
+  uint64_t z[N / 2];  // z = y - kTailY
   uint32_t all = 0xffffffffu;  // AND of the words: bit 31 set iff every z < 0
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
+  for (int e = 0; e < N / 2; ++e) {
     z[e] = f2_fma(f2_pack(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1])), c1, c0);
     all &= static_cast<uint32_t>(z[e]) & static_cast<uint32_t>(z[e] >> 32);
   }
   if (__all_sync(0xffffffffu, (all >> 31) != 0)) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
+    for (int e = 0; e < N / 2; ++e) {
       const float2 zz = f2_unpack(z[e]);
       const uint64_t w = f2_pack(ex2_approx(zz.x), ex2_approx(zz.y));
       uint64_t t = f2_fma(w, f2_splat(kTailC * kTailC * kTailC), f2_splat(-kTailC * kTailC));
@@ -293,7 +294,7 @@ __device__ __forceinline__ void sigmoid32(uint32_t (&a)[32], float scale_l2e, fl
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
+    for (int e = 0; e < N / 2; ++e) {
       const float2 yy = f2_unpack(f2_fma(z[e], f2_splat(1.0f), f2_splat(kTailY)));
       const uint64_t u = f2_pack(ex2_approx(-fabsf(yy.x)), ex2_approx(-fabsf(yy.y)));
       const uint64_t t = poly_t2(u);
@@ -311,15 +312,21 @@ __device__ __forceinline__ void sigmoid32(uint32_t (&a)[32], float scale_l2e, fl
   }
 }
 
+template <bool SLOPE>
+__device__ __forceinline__ void sigmoid32(uint32_t (&a)[32], float scale_l2e, float neg_log2n, float* slope) {
+  sigmoid_n<SLOPE, 32>(a, scale_l2e, neg_log2n, slope);
+}
+
 // Scores that must not count: the columns at or past `valid` (keys beyond
 // the sequence) and every column of a row that is not a valid token. Set to
 // -inf, their weight and its derivative come out exactly 0 on either form,
 // and they take no part in the warp's choice of form, so values in padded
 // rows never change the bits of a valid output.
-__device__ __forceinline__ void mask_scores(uint32_t (&a)[32], int valid, bool row_ok) {
-  if (valid >= 32 && row_ok) return;
+template <int N>
+__device__ __forceinline__ void mask_scores(uint32_t (&a)[N], int valid, bool row_ok) {
+  if (valid >= N && row_ok) return;
 #pragma unroll
-  for (int e = 0; e < 32; ++e)
+  for (int e = 0; e < N; ++e)
     if (!row_ok || e >= valid) a[e] = 0xff800000u;
 }
 
