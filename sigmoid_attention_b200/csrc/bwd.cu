@@ -51,10 +51,10 @@ struct BwdCfg {
   static constexpr int BM = kBwdItemRows;   // 128 rows per item
   static constexpr int BN = bwd_col_block(KV, D);
   // Epilogue column groups (warps per lane quadrant) and chunk width: 8
-  // epilogue warps on 32-column chunks. (16 warps on 16-column chunks for
-  // dK/dV at D = 128, at 88 registers each, measured slower: 0.918 -> 0.984 ms
-  // on the dense d = 128 workload.)
-  static constexpr int GROUPS = 2;
+  // epilogue warps on 32-column chunks, 16 for dQ at D = 64. (16 warps on
+  // 16-column chunks for dK/dV at D = 128, at 88 registers each, measured
+  // slower: 0.918 -> 0.984 ms on the dense d = 128 workload.)
+  static constexpr int GROUPS = (D == 64) ? 4 : 2;
   static constexpr int CW = 32;
   static constexpr int NCH = BN / CW;       // chunks per block
   static constexpr int CPW = NCH / GROUPS;  // chunks per epilogue warp
@@ -99,7 +99,7 @@ struct BwdCfg {
   static constexpr int WARPS = (EPI_WARPS + 1 + ISSUERS + 3) / 4 * 4 < 16 ? 16 : (EPI_WARPS + 1 + ISSUERS + 3) / 4 * 4;
   static constexpr int THREADS = WARPS * 32;
   static constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
-  static constexpr int OTHER_REGS = WARPS > 16 ? 56 : 64;
+  static constexpr int OTHER_REGS = WARPS > 20 ? 48 : WARPS > 16 ? 56 : 64;
   static constexpr int EPI_REGS =
       ((LAUNCH_REGS * WARPS - OTHER_REGS * (WARPS - EPI_WARPS)) / EPI_WARPS) / 8 * 8 > 184
           ? 184
@@ -320,49 +320,50 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       const bool in_range = rm.writes(row, n);
       const bool valid_row = row < (KV ? range_keys(n, kr) : n);
       const size_t row_off = rm.offset(item, PACKED ? item.bh % H : 0, row, D);
-      // 32-column chunks of the accumulators: A1 (-> out1, times scale), then
-      // A2 (-> out2) for dK/dV; column group g takes chunks g, g + G, ...
+      // Chunks of RW accumulator columns (32, or 16 where the column groups
+      // outnumber the 32-column chunks): A1 (-> out1, times scale), then A2
+      // (-> out2) for dK/dV; column group g takes chunks g, g + G, ...
       // Each chunk is copied out and packed to bf16 at once, so the
       // accumulators are released before the (slower) global stores.
-      constexpr int kChunks = (KV ? 2 : 1) * (D / 32);
+      constexpr int kCols = (KV ? 2 : 1) * D;
+      constexpr int RW = kCols / G >= 32 ? 32 : 16;
+      constexpr int kChunks = kCols / RW;
       constexpr int kPer = kChunks / G;
       static_assert(kPer * G == kChunks, "accumulator chunks");
       // bf16 pairs, or (F32OUT) the fp32 values themselves
-      uint32_t packed[kPer][F32OUT ? 32 : 16];
+      constexpr int kWords = F32OUT ? RW : RW / 2;
+      uint32_t packed[kPer][kWords];
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
         const int c = g + G * i;
-        const bool second = c >= D / 32;
-        const int col = (second ? c - D / 32 : c) * 32;
+        const bool second = c >= D / RW;
+        const int col = (second ? c - D / RW : c) * RW;
         const float mul = (second ? 1.0f : scale) * (valid_row ? 1.0f : 0.0f);
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v);
+        uint32_t v[RW];
+        tmem_ld_async(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v);
+        tmem_ld_wait(v);
         if constexpr (F32OUT) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) packed[i][e] = valid_row ? __float_as_uint(__uint_as_float(v[e]) * mul) : 0u;
+          for (int e = 0; e < RW; ++e) packed[i][e] = valid_row ? __float_as_uint(__uint_as_float(v[e]) * mul) : 0u;
         } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            packed[i][e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+          for (int e = 0; e < RW / 2; ++e)
+            packed[i][e] = valid_row ? pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul)
+                                     : 0u;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.acc_empty);
-      if (in_range) {
+      if (in_range) {  // rows past the valid ones get zeros
 #pragma unroll
         for (int i = 0; i < kPer; ++i) {
           const int c = g + G * i;
-          const bool second = c >= D / 32;
-          const int col = (second ? c - D / 32 : c) * 32;
+          const bool second = c >= D / RW;
+          const int col = (second ? c - D / RW : c) * RW;
           void* out = second ? out2 : out1;
-          if constexpr (F32OUT) {
-            store_row_f32(static_cast<float*>(out) + row_off + col, packed[i]);  // zeros already for padded rows
-          } else if (valid_row) {
-            store_row64B(static_cast<__nv_bfloat16*>(out) + row_off + col, packed[i]);
-          } else {
-            store_zero32(static_cast<__nv_bfloat16*>(out) + row_off + col);
-          }
+          const size_t off = (row_off + col) * (F32OUT ? 4 : 2);
+          store_words(static_cast<uint8_t*>(out) + off, packed[i]);
         }
       }
     }

@@ -414,6 +414,26 @@ __device__ __forceinline__ void store_row64B(void* dst, const uint32_t (&w)[16])
   }
 }
 
+// Store NW 32-bit words (32, 64 or 128 bytes of one row) at dst, 16-byte
+// aligned; 32-byte stores when dst is 32-byte aligned (warp-uniform).
+template <int NW>
+__device__ __forceinline__ void store_words(void* dst, const uint32_t (&w)[NW]) {
+  static_assert(NW % 8 == 0, "whole 32-byte pieces");
+  if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+#pragma unroll
+    for (int h = 0; h < NW / 8; ++h)
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                       reinterpret_cast<uint8_t*>(dst) + 32 * h),
+                   "r"(w[8 * h]), "r"(w[8 * h + 1]), "r"(w[8 * h + 2]), "r"(w[8 * h + 3]), "r"(w[8 * h + 4]),
+                   "r"(w[8 * h + 5]), "r"(w[8 * h + 6]), "r"(w[8 * h + 7])
+                   : "memory");
+  } else {
+    uint4* p = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < NW / 4; ++q) p[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
 // Convert 32 fp32 accumulator values (times `mul`) to bf16 and store them.
 __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul) {
   uint32_t w[16];
