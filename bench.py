@@ -230,8 +230,9 @@ def run_reference(args, w):
 
 
 def _run_calls(calls, stream, ev=None):
-    """One step: the forward, dQ and dK/dV calls, with an event before each
-    call and after the last when `ev` (four CUDA events) is given."""
+    """One step: the forward, dQ and dK/dV calls (or the forward and the
+    whole-backward call), with an event before each call and after the last
+    when `ev` (len(calls) + 1 CUDA events) is given."""
     for i, call in enumerate(calls):
         if ev is not None:
             ev[i].record(stream)
@@ -246,7 +247,8 @@ def _check_status(sa, ws, stream):
         raise SystemExit(f"kernel reported status {st} at site {site}")
 
 
-def _device_steps(calls, stream, steps, warmup, flush_buf=None, sync_ranks=None, check=None, sampler=None):
+def _device_steps(calls, stream, steps, warmup, flush_buf=None, sync_ranks=None, check=None, sampler=None,
+                  names=("fwd", "bwd_dq", "bwd_dkdv")):
     """Device time of each call over `steps` timed steps after `warmup`
     untimed ones: CUDA events on the launching stream, a synchronize (and a
     barrier over ranks, when given) on both sides of the timed region, and an
@@ -262,7 +264,7 @@ def _device_steps(calls, stream, steps, warmup, flush_buf=None, sync_ranks=None,
             flush_buf.zero_()
     if check is not None:
         check()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
     if sync_ranks is not None:
         sync_ranks()
     torch.cuda.synchronize()
@@ -276,14 +278,27 @@ def _device_steps(calls, stream, steps, warmup, flush_buf=None, sync_ranks=None,
         sync_ranks()
     if check is not None:
         check()
-    per_kernel = {"fwd": [], "bwd_dq": [], "bwd_dkdv": []}
+    per_kernel = {name: [] for name in names}
     step_ms = []
     for ev in events:
-        per_kernel["fwd"].append(ev[0].elapsed_time(ev[1]))
-        per_kernel["bwd_dq"].append(ev[1].elapsed_time(ev[2]))
-        per_kernel["bwd_dkdv"].append(ev[2].elapsed_time(ev[3]))
-        step_ms.append(ev[0].elapsed_time(ev[3]))
+        for i, name in enumerate(names):
+            per_kernel[name].append(ev[i].elapsed_time(ev[i + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[-1]))
     return per_kernel, step_ms
+
+
+def _fused_backward(per_kernel_sep, fused_calls, stream, steps, warmup, flush_buf, check, flops_fwd, flops_bwd):
+    """The same step with the whole-backward call (sigattn_bwd: the dQ and
+    dK/dV kernels overlapped) instead of the two backward calls, timed the
+    same way right after the separate-call steps."""
+    per_kernel, step_ms = _device_steps(fused_calls, stream, steps, warmup, flush_buf, check=check,
+                                        names=("fwd", "bwd"))
+    bwd_ms = float(np.mean(per_kernel["bwd"]))
+    sep_ms = float(np.mean(per_kernel_sep["bwd_dq"])) + float(np.mean(per_kernel_sep["bwd_dkdv"]))
+    return {"value": (flops_fwd + flops_bwd) / (np.mean(step_ms) / 1e3) / 1e12,
+            "bwd_ms": bwd_ms, "bwd_tflops": flops_bwd / (bwd_ms / 1e3) / 1e12,
+            "bwd_speedup_vs_two_calls": sep_ms / bwd_ms,
+            "step": "sigattn_fwd + sigattn_bwd (dQ and dK/dV kernels overlapped)"}
 
 
 def side_workloads(names, dev, steps: int, warmup: int) -> dict:
@@ -312,13 +327,18 @@ def side_workloads(names, dev, steps: int, warmup: int) -> dict:
                                             check=lambda: _check_status(sa, ws, stream))
         f_fwd, f_bwd = w.fwd_flops(), w.bwd_flops()
         ms = {kname: float(np.mean(v_)) for kname, v_ in per_kernel.items()}
+        fused_calls = (calls[0], lambda: sa.sigattn_bwd(qd, kd, vd, dod, dq, dk, dv, lens, ws, stream))
         out[name] = {"value": (f_fwd + f_bwd) / (np.mean(step_ms) / 1e3) / 1e12,
                      "fwd_tflops": f_fwd / (ms["fwd"] / 1e3) / 1e12,
                      "bwd_tflops": f_bwd / ((ms["bwd_dq"] + ms["bwd_dkdv"]) / 1e3) / 1e12,
-                     "ms": ms, "steps": steps}
+                     "ms": ms, "steps": steps,
+                     "step_fused": _fused_backward(per_kernel, fused_calls, stream, steps, warmup, flush_buf,
+                                                   lambda: _check_status(sa, ws, stream), f_fwd, f_bwd)}
         del qd, kd, vd, dod, o, dq, dk, dv, ws
     if "pad_sweep_p00" in out and "pad_sweep_p75" in out:
         out["p75_over_p00"] = out["pad_sweep_p75"]["value"] / out["pad_sweep_p00"]["value"]
+        out["p75_over_p00_fused"] = (out["pad_sweep_p75"]["step_fused"]["value"] /
+                                     out["pad_sweep_p00"]["step_fused"]["value"])
     return out
 
 
@@ -497,6 +517,15 @@ def run_gpu(args, w):
     clocks = ClockSampler(local)
     per_kernel, step_ms = _device_steps(calls, stream, args.steps, args.warmup, scratch, sync_ranks,
                                         lambda: _check_status(sa, ws, stream), clocks)
+    step_fused = None
+    if not packed:
+        fused_calls = (calls[0], lambda: sa.sigattn_bwd(qd, kd, vd, dod, dq, dk, dv, lens, ws, stream))
+        step_fused = _fused_backward(per_kernel, fused_calls, stream, args.steps, args.warmup, scratch,
+                                     lambda: _check_status(sa, ws, stream), flops_fwd, flops_bwd)
+        if world > 1:  # whole-job figures: the slowest rank's time
+            for key in ("value", "bwd_tflops"):
+                step_fused[key] = world / reduce_max(world / step_fused[key], world, dev)
+            step_fused.pop("bwd_speedup_vs_two_calls")
     total_s = reduce_max(sum(step_ms) / 1e3, world, dev)
     fwd_s = reduce_max(sum(per_kernel["fwd"]) / 1e3, world, dev)
     bwd_s = reduce_max((sum(per_kernel["bwd_dq"]) + sum(per_kernel["bwd_dkdv"])) / 1e3, world, dev)
@@ -563,8 +592,7 @@ def run_gpu(args, w):
             else:
                 lc = lens[r0:r1]
                 sa.sigattn_fwd(qc, kc, vc, oc, lc, ws, stream)
-                sa.sigattn_bwd_dq(qc, kc, vc, dc, dqc, lc, ws, stream)
-                sa.sigattn_bwd_dkdv(qc, kc, vc, dc, dkc, dvc, lc, ws, stream)
+                sa.sigattn_bwd(qc, kc, vc, dc, dqc, dkc, dvc, lc, ws, stream)
             computed[c].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(computed[c])
@@ -632,12 +660,14 @@ def run_gpu(args, w):
         "fwd_frac_of_peak": fwd_tflops / peak, "bwd_frac_of_peak": bwd_tflops / peak,
         "frac_of_spec_2250": {"fwd": fwd_tflops / 2250.0, "bwd": bwd_tflops / 2250.0},
         "kernels": kernels,
+        "step_fused": step_fused,
         "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "peak_source": f"bf16_tflops ({peaks['source']}, burst)",
                      "traffic": _traffic(dominant, w.name)},
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps,
-                "schedule": f"{len(rows)} chunks of whole sequences; host-to-device copies, the three calls and "
+                "schedule": f"{len(rows)} chunks of whole sequences; host-to-device copies, the calls "
+                            f"({'three varlen calls' if packed else 'sigattn_fwd + sigattn_bwd'}) and "
                             "device-to-host copies on three streams",
                 "pcie_gbs": pcie, "bound": e2e_bound, "frac_of_bound": e2e_value / e2e_bound,
                 "bound_source": "larger copy direction per step at the measured both-ways pinned copy rate"},

@@ -112,6 +112,26 @@ SIGATTN_API int sigattn_bwd_dkdv(const void* q, const void* k, const void* v, co
                      const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* The whole backward pass in one call: dq as sigattn_bwd_dq, dk and dv as
+ * sigattn_bwd_dkdv, with identical results (the same kernels, each with one
+ * owner per output block and a fixed summation order). The two gradients
+ * depend only on q, k, v and dout (sec. 2B/2C: no row statistics of the
+ * forward pass are needed), so one plan launch builds both work lists and
+ * the dK/dV kernel takes each SM as soon as the dQ kernel's CTA on it has
+ * finished, instead of after the last of them: the end of the dQ kernel,
+ * where fewer work items than SMs remain, overlaps the start of the dK/dV
+ * kernel. The call's last kernel completes only after both have, so later
+ * work in the stream sees all three outputs.
+ *  - workspace: at least sigattn_bwd_workspace_size(B, H, Lmax, d) bytes
+ *    (two work lists); 16-byte aligned and zeroed once, as for every call.
+ *    Errors of both kernels go to its sticky error word.
+ *  - dq, dk, dv must not overlap each other or the inputs.
+ * Returns 0 from sigattn_bwd_workspace_size if the sizes are out of range. */
+SIGATTN_API size_t sigattn_bwd_workspace_size(int B, int H, int Lmax, int d);
+SIGATTN_API int sigattn_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
+                            void* dv, const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
 /* Key ranges: the padded-layout calls restricted to the keys at positions
  * [key_begin, key_begin + key_count) of every sequence, for attention whose
  * keys are split over several calls or GPUs (sequence sharding). Because each

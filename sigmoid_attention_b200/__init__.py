@@ -20,7 +20,8 @@ import torch
 
 __all__ = [
     "SigattnError", "library", "library_path", "sigattn_version", "sigattn_status_str", "sigattn_block_rows",
-    "sigattn_workspace_size", "sigattn_fwd", "sigattn_fwd_noalloc", "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
+    "sigattn_workspace_size", "sigattn_bwd_workspace_size", "sigattn_fwd", "sigattn_fwd_noalloc", "sigattn_bwd",
+    "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
     "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "sigattn_eval_sigmoid", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
     "sigattn_fwd_varlen", "sigattn_bwd_dq_varlen", "sigattn_bwd_dkdv_varlen",
     "sigattn_fwd_partial", "sigattn_bwd_dq_partial", "sigattn_bwd_dkdv_range", "sigattn_cast_bf16",
@@ -73,6 +74,10 @@ def library():
         lib.sigattn_bwd_dq.argtypes = [_vp] * 6 + [_i] * 4 + [_vp, _sz, _vp]
         lib.sigattn_bwd_dkdv.restype = _i
         lib.sigattn_bwd_dkdv.argtypes = [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]
+        lib.sigattn_bwd_workspace_size.restype = _sz
+        lib.sigattn_bwd_workspace_size.argtypes = [_i] * 4
+        lib.sigattn_bwd.restype = _i
+        lib.sigattn_bwd.argtypes = [_vp] * 8 + [_i] * 4 + [_vp, _sz, _vp]
         lib.sigattn_fwd_varlen.restype = _i
         lib.sigattn_fwd_varlen.argtypes = [_vp] * 5 + [_i] * 5 + [_vp, _sz, _vp]
         lib.sigattn_bwd_dq_varlen.restype = _i
@@ -149,9 +154,14 @@ def sigattn_workspace_size(B: int, H: int, Lmax: int, d: int) -> int:
     return library().sigattn_workspace_size(B, H, Lmax, d)
 
 
+def sigattn_bwd_workspace_size(B: int, H: int, Lmax: int, d: int) -> int:
+    return library().sigattn_bwd_workspace_size(B, H, Lmax, d)
+
+
 def make_workspace(B: int, H: int, Lmax: int, d: int, device=None) -> torch.Tensor:
-    """A zero-initialised workspace (uint8 CUDA tensor) big enough for any call."""
-    n = sigattn_workspace_size(B, H, Lmax, d)
+    """A zero-initialised workspace (uint8 CUDA tensor) big enough for any
+    call, ``sigattn_bwd`` (two work lists) included."""
+    n = max(sigattn_workspace_size(B, H, Lmax, d), sigattn_bwd_workspace_size(B, H, Lmax, d))
     if n == 0:
         raise SigattnError("sigattn_workspace_size", 2)
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
@@ -196,6 +206,16 @@ def sigattn_bwd_dkdv(q, k, v, dout, dk, dv, lengths, workspace, stream=None) -> 
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dk, "dk"), _dev(dv, "dv"),
         _dev(lengths, "lengths", torch.int32), B, H, L, d, _dev(workspace, "workspace", torch.uint8),
         workspace.numel(), _stream_ptr(stream)))
+
+
+def sigattn_bwd(q, k, v, dout, dq, dk, dv, lengths, workspace, stream=None) -> None:
+    """dQ, dK and dV in one call (the two backward kernels overlapped; results
+    identical to sigattn_bwd_dq + sigattn_bwd_dkdv)."""
+    B, H, L, d = _dims(q)
+    _check("sigattn_bwd", library().sigattn_bwd(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"),
+        _dev(dv, "dv"), _dev(lengths, "lengths", torch.int32), B, H, L, d,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
 
 
 def sigattn_fwd_partial(q, k, v, o_partial, lengths, key_begin: int, workspace, stream=None) -> None:
@@ -339,8 +359,7 @@ def backward(q, k, v, dout, lengths, workspace=None, stream=None):
     if workspace is None:
         workspace = make_workspace(B, H, L, d, q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    sigattn_bwd_dq(q, k, v, dout, dq, lengths, workspace, stream)
-    sigattn_bwd_dkdv(q, k, v, dout, dk, dv, lengths, workspace, stream)
+    sigattn_bwd(q, k, v, dout, dq, dk, dv, lengths, workspace, stream)
     return dq, dk, dv
 
 
@@ -359,8 +378,9 @@ def _check_device_status(fn: str, workspace, check: bool) -> None:
 
 
 class SigmoidAttentionFunction(torch.autograd.Function):
-    """Autograd wrapper: forward with ``sigattn_fwd``, backward with the two
-    backward calls (a drop-in for softmax attention over padded batches)."""
+    """Autograd wrapper: forward with ``sigattn_fwd``, backward with
+    ``sigattn_bwd`` (dQ, dK and dV in one call; a drop-in for softmax
+    attention over padded batches)."""
 
     @staticmethod
     def forward(ctx, q, k, v, lengths, check=False):

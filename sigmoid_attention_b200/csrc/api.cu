@@ -26,12 +26,15 @@ cudaError_t launch_fwd(int d, bool packed, bool f32out, const CUtensorMap& tq, c
                        cudaStream_t stream);
 cudaError_t launch_softmax_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
                                int B, int H, int L, int num_sms, cudaStream_t stream);
+cudaError_t launch_prep_bwd(const int* lengths, int B, int H, int L, int* ws_dq, int* ws_dkdv, cudaStream_t stream);
 cudaError_t launch_bwd_dq(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tdo,
                           const CUtensorMap& tk, const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L,
-                          KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream);
+                          KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream,
+                          const BwdLink& link = BwdLink{});
 cudaError_t launch_bwd_dkdv(int d, bool packed, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                             const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int out_rows, int Lmax,
-                            KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream);
+                            KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream,
+                            const BwdLink& link = BwdLink{});
 void set_last_error(const char* msg);
 }  // namespace sigattn
 
@@ -252,6 +255,49 @@ int dkdv_padded(const void* q, const void* k, const void* v, const void* dout, v
       launch_bwd_dkdv(d, false, tk, tv, tq, tdo, dk, dv, ws, B, H, kr.count, Lmax, kr, info.num_sms, lengths, s));
 }
 
+// Bytes of one plan region (header and work list), rounded up to 256 so that
+// the second region of a whole-backward workspace stays aligned.
+size_t plan_region_bytes(int B, int H, int Lmax) {
+  const size_t n = static_cast<size_t>(kHeaderWords) * 4 + static_cast<size_t>(max_items(B, H, Lmax)) * 16;
+  return (n + 255) / 256 * 256;
+}
+
+// dQ, dK and dV in one call: one plan launch builds both work lists (dQ's in
+// the workspace's first region, dK/dV's in the second), then the dQ kernel
+// and the dK/dV kernel, which takes SMs as the dQ kernel's CTAs finish and
+// completes after it (bwd.cu). Errors of both go to the first header.
+int bwd_padded(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk, void* dv,
+               const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  if (workspace_bytes < sigattn_bwd_workspace_size(B, H, Lmax, d)) return SIGATTN_ERR_INVALID_ARG;
+  DeviceInfo info;
+  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  if (st != SIGATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return SIGATTN_ERR_INVALID_ARG;
+  const int cb = bwd_col_block(true, d);
+  CUtensorMap tq, tk, tv, tdo, tq_c, tdo_c;
+  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) || !make_map(&tv, v, B * H, Lmax, d) ||
+      !make_map(&tdo, dout, B * H, Lmax, d) || !make_map(&tq_c, q, B * H, Lmax, d, cb) ||
+      !make_map(&tdo_c, dout, B * H, Lmax, d, cb))
+    return map_failure();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws_dq = static_cast<int*>(workspace);
+  int* ws_dkdv = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan_region_bytes(B, H, Lmax));
+  const KeyRange all{0, Lmax};
+  st = cuda_status(launch_prep_bwd(lengths, B, H, Lmax, ws_dq, ws_dkdv, s));
+  if (st == SIGATTN_OK)
+    st = cuda_status(launch_bwd_dq(d, false, false, tq, tdo, tk, tv, dq, ws_dq, B, H, Lmax, all, info.num_sms,
+                                   lengths, s));
+  if (st != SIGATTN_OK) return st;
+  BwdLink link;
+  link.err = ws_dq;
+  link.overlap = true;
+  return cuda_status(launch_bwd_dkdv(d, false, tk, tv, tq_c, tdo_c, dk, dv, ws_dkdv, B, H, Lmax, Lmax, all,
+                                     info.num_sms, lengths, s, link));
+}
+
 }  // namespace
 
 namespace sigattn {
@@ -302,6 +348,17 @@ int sigattn_block_rows(int kind) {
 size_t sigattn_workspace_size(int B, int H, int Lmax, int d) {
   if (check_sizes(B, H, Lmax, d) != SIGATTN_OK) return 0;
   return static_cast<size_t>(kHeaderWords) * 4 + static_cast<size_t>(max_items(B, H, Lmax)) * 16;
+}
+
+size_t sigattn_bwd_workspace_size(int B, int H, int Lmax, int d) {
+  if (check_sizes(B, H, Lmax, d) != SIGATTN_OK) return 0;
+  return 2 * plan_region_bytes(B, H, Lmax);
+}
+
+int sigattn_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk, void* dv,
+                const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  return bwd_padded(q, k, v, dout, dq, dk, dv, lengths, B, H, Lmax, d, workspace, workspace_bytes, stream);
 }
 
 int sigattn_fwd(const void* q, const void* k, const void* v, void* o, const int32_t* lengths, int B, int H,

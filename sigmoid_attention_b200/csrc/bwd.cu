@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_r1, const __grid_constant__ CUtensorMap tm_r2,
                const __grid_constant__ CUtensorMap tm_c1, const __grid_constant__ CUtensorMap tm_c2,
                void* __restrict__ out1, void* __restrict__ out2, int* __restrict__ ws, int H, int L, KeyRange kr,
-               const int* __restrict__ fill_lengths, int B, int len_bound, int fill_parts) {
+               const int* __restrict__ fill_lengths, int B, int len_bound, int fill_parts, int* __restrict__ err,
+               int overlap) {
   using C = BwdCfg<D, KV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ BwdBarriers<C::ST1, C::ST2> bar;
@@ -142,7 +143,6 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = &bar.abort;
-  grid_dep_launch();  // the padded-row fill kernel may start beside this one
   constexpr int kProducerWarp = C::EPI_WARPS;
   constexpr int kSWarp = C::EPI_WARPS + 1;
   constexpr int kDPWarp = C::EPI_WARPS + 2;
@@ -195,11 +195,17 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     for (int i = threadIdx.x; i < C::ZBUF / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
-  // The plan is written by the kernel before this one in the stream.
-  grid_dep_wait();
+  // The plan is written by the kernel before this one in the stream. With
+  // `overlap` (the dK/dV kernel of a whole-backward call) the kernel before is
+  // the dQ kernel, which reads nothing this one writes and whose CTAs launch
+  // this one only after their own wait for the plan: the wait moves to the end
+  // (so that this grid completes after the dQ grid) and the kernel takes SMs
+  // as the dQ kernel's CTAs leave them.
+  if (!overlap) grid_dep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_dep_launch();
   const uint32_t tmem = bar.tmem_base;
   const int count = ws[kHdrCount];
   const RowMap<PACKED> rm{H, L};
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     uint32_t ist = 0, iph = 0;
     while (ok) {
       Item item;
-      if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 220))) break;
+      if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, err, 220))) break;
       __syncwarp();
       ring_release(bar.ring, ist, iph, lane == 0);
       if (item.n < 0) break;
@@ -244,7 +250,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         uint32_t pk[KV ? CPW : 1][CW / 2];
         {
           uint32_t sv[CPW][CW];
-          if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, ws, 221))) break;
+          if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, err, 221))) break;
           s_ph ^= 1;
           tc_fence_after();
 #pragma unroll
@@ -267,7 +273,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           }
         }
         if (KV) {
-          if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, ws, 223))) break;
+          if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, err, 223))) break;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         uint32_t dp[CPW][CW];
         const uint32_t tXDP = xb ? tXDP1 : tXDP0;
         uint64_t* xdp_read = &bar.xdp_read[xb];
-        if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, ws, 222))) break;
+        if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, err, 222))) break;
         dp_ph[xb] ^= 1;
         if (++xb == static_cast<uint32_t>(C::NXDP)) xb = 0;
         tc_fence_after();
@@ -294,7 +300,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(xdp_read);
-        if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, ws, 224))) break;
+        if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, err, 224))) break;
         free_ph ^= 1;
         tc_fence_after();
 #pragma unroll
@@ -302,9 +308,11 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const uint32_t(&dpc)[CW] = dp[c];
           uint32_t dk[CW / 2];
 #pragma unroll
-          for (int e = 0; e < CW / 2; ++e)
-            dk[e] = pack_bf16x2(__uint_as_float(dpc[2 * e]) * sp[c][2 * e],
-                                __uint_as_float(dpc[2 * e + 1]) * sp[c][2 * e + 1]);
+          for (int e = 0; e < CW / 2; ++e) {
+            const float2 ds = f2_unpack(f2_mul(f2_pack(__uint_as_float(dpc[2 * e]), __uint_as_float(dpc[2 * e + 1])),
+                                               f2_pack(sp[c][2 * e], sp[c][2 * e + 1])));
+            dk[e] = pack_bf16x2(ds.x, ds.y);
+          }
           tmem_st(tmem + lane_off + C::TM_DS + (g * CPW + c) * (CW / 2), dk);
           tmem_st_wait();
           tc_fence_before();
@@ -313,7 +321,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         }
       }
       if (!ok) break;
-      if (!(ok = mbar_wait(&bar.acc_full, aph, abort_flag, ws, 225))) break;
+      if (!(ok = mbar_wait(&bar.acc_full, aph, abort_flag, err, 225))) break;
       aph ^= 1;
       tc_fence_after();
       const int row = item.blk * C::BM + r;
@@ -403,7 +411,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         };
         while (ok) {
           const Item item = next_item(ws, claimed, count);
-          if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, ws, 200))) break;
+          if (!(ok = ring_publish(bar.ring, ist, iph, item, abort_flag, err, 200))) break;
           if (item.n < 0) break;
           const int n = item.n;
           const int hd = PACKED ? item.bh % H : 0;
@@ -412,7 +420,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
             issue_fill();
             fill_u = atomicAdd(ws + kHdrFill, 1);
           }
-          if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, ws, 201))) break;
+          if (!(ok = mbar_wait(&bar.r_empty, rph ^ 1, abort_flag, err, 201))) break;
           mbar_arrive_expect_tx(&bar.r_full, 2 * C::TILE_R);
           for (int c = 0; c < D / 64; ++c) {
             const int ry = rm.y(item, hd, item.blk * C::BM), rz = rm.z(item, item.blk * C::BM);
@@ -424,14 +432,14 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           for (int j = 0; j < nb; ++j) {
             // Claim the CTA's next item two column blocks before this one ends.
             if (j == max(0, nb - 2)) claimed = atomicAdd(ws + kHdrNext, 1);
-            if (!(ok = mbar_wait(&bar.c1_empty[s1], p1 ^ 1, abort_flag, ws, 202))) break;
+            if (!(ok = mbar_wait(&bar.c1_empty[s1], p1 ^ 1, abort_flag, err, 202))) break;
             mbar_arrive_expect_tx(&bar.c1_full[s1], C::TILE_C);
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(smem + C::OFF_C1 + s1 * C::TILE_C + c * C::BOX_C, &tm_c1, &bar.c1_full[s1], c * 64,
                           rm.y(item, hd, j * C::BN), rm.z(item, j * C::BN));
             c1_last[s1] = static_cast<int>(p1);
             if (++s1 == C::ST1) { s1 = 0; p1 ^= 1; }
-            if (!(ok = mbar_wait(&bar.c2_empty[s2], p2 ^ 1, abort_flag, ws, 203))) break;
+            if (!(ok = mbar_wait(&bar.c2_empty[s2], p2 ^ 1, abort_flag, err, 203))) break;
             mbar_arrive_expect_tx(&bar.c2_full[s2], C::TILE_C);
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(smem + C::OFF_C2 + s2 * C::TILE_C + c * C::BOX_C, &tm_c2, &bar.c2_full[s2], c * 64,
@@ -473,21 +481,21 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         uint32_t ist = 0, iph = 0;
         while (ok) {
           Item item;
-          if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 210))) break;
+          if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, err, 210))) break;
           ring_release(bar.ring, ist, iph, true);
           if (item.n < 0) break;
           const int n = item.n;
           const int nb = ceil_div(work_cols(KV ? kKindDkdv : kKindDq, n, kr), C::BN);
-          if (!(ok = mbar_wait(&bar.r_full, rph, abort_flag, ws, 211))) break;
+          if (!(ok = mbar_wait(&bar.r_full, rph, abort_flag, err, 211))) break;
           rph ^= 1;
           for (int j = 0; j < nb; ++j) {
-            if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 212))) break;
+            if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, err, 212))) break;
             // The region is free once the epilogue has copied out the block that
             // last used it (block j-1, or j-2 with two dP regions).
             uint64_t* xread = is_dp ? &bar.xdp_read[xb] : &bar.xs_read;
             uint64_t* xfull = is_dp ? &bar.xdp_full[xb] : &bar.xs_full;
             const uint32_t d_tmem = tmem + (is_dp ? (xb ? C::TM_XDP1 : C::TM_XDP) : C::TM_XS);
-            if (!(ok = mbar_wait(xread, read_ph[xb] ^ 1, abort_flag, ws, 213))) break;
+            if (!(ok = mbar_wait(xread, read_ph[xb] ^ 1, abort_flag, err, 213))) break;
             read_ph[xb] ^= 1;
             tc_fence_after();
             const uint64_t b0 = d_c + st * kTileC;
@@ -506,7 +514,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         }
         int never = 0;
         mma_commit(&bar.drain[is_dp ? 1 : 0]);
-        mbar_wait(&bar.drain[is_dp ? 1 : 0], 0, &never, ws, 219);
+        mbar_wait(&bar.drain[is_dp ? 1 : 0], 0, &never, err, 219);
       }
     } else if (warp == kA1Warp || warp == kA2Warp) {
       // -------------------------- issuers of A1 += dS C1 and (dK/dV) A2 += P C2
@@ -529,20 +537,20 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         uint32_t ist = 0, iph = 0;
         while (ok) {
           Item item;
-          if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, ws, 210))) break;
+          if (!(ok = ring_read(bar.ring, ist, iph, &item, abort_flag, err, 210))) break;
           ring_release(bar.ring, ist, iph, true);
           if (item.n < 0) break;
           const int n = item.n;
           const int nb = ceil_div(work_cols(KV ? kKindDkdv : kKindDq, n, kr), C::BN);
           for (int j = 0; ok && j < nb; ++j) {
-            if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, ws, 231))) break;
+            if (!(ok = mbar_wait(&cfull[st], cph, abort_flag, err, 231))) break;
             const uint64_t b0 = d_cmn + st * kTileC;
             for (int q = 0; q < C::NCH; ++q) {
-              if (!(ok = mbar_wait(&full[q], fph[q], abort_flag, ws, 232))) break;
+              if (!(ok = mbar_wait(&full[q], fph[q], abort_flag, err, 232))) break;
               fph[q] ^= 1;
               const bool first = (j == 0 && q == 0);
               if (first) {
-                if (!(ok = mbar_wait(&bar.acc_empty, aph ^ 1, abort_flag, ws, 233))) break;
+                if (!(ok = mbar_wait(&bar.acc_empty, aph ^ 1, abort_flag, err, 233))) break;
                 aph ^= 1;
               }
               tc_fence_after();
@@ -563,7 +571,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         }
         int never = 0;
         mma_commit(&bar.drain[second ? 3 : 2]);
-        mbar_wait(&bar.drain[second ? 3 : 2], 0, &never, ws, 239);
+        mbar_wait(&bar.drain[second ? 3 : 2], 0, &never, err, 239);
       }
     }
   }
@@ -591,12 +599,14 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  if (overlap) grid_dep_wait();
 }
 
 template <int D, bool KV, bool PACKED, bool F32OUT>
 cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const CUtensorMap& c1,
                             const CUtensorMap& c2, void* out1, void* out2, int* ws, int B, int H, int L, KeyRange kr,
-                            int num_sms, const int* fill_lengths, int len_bound, cudaStream_t stream) {
+                            int num_sms, const int* fill_lengths, int len_bound, cudaStream_t stream,
+                            const BwdLink& link) {
   using C = BwdCfg<D, KV>;
   static PerDeviceOnce attr;
   const cudaError_t e = attr.run([] {
@@ -618,7 +628,8 @@ cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const 
   const int grid = static_cast<int>(std::min<long long>(num_sms, max_items));
   const int parts = zero_fill_parts(static_cast<long long>(B) * H, num_sms);
   return launch_programmatic(bwd_kernel<D, KV, PACKED, F32OUT>, dim3(grid), dim3(C::THREADS), C::SMEM_ALLOC, stream,
-                             r1, r2, c1, c2, out1, out2, ws, H, L, kr, fill_lengths, B, len_bound, parts);
+                             r1, r2, c1, c2, out1, out2, ws, H, L, kr, fill_lengths, B, len_bound, parts,
+                             link.err != nullptr ? link.err : ws, link.overlap ? 1 : 0);
 }
 
 // fill_lengths: the padded layout's lengths, so that the kernel zeroes the
@@ -627,26 +638,27 @@ cudaError_t launch_bwd_impl(const CUtensorMap& r1, const CUtensorMap& r2, const 
 // ({0, L} for whole sequences); f32out: dQ as the fp32 partial sum over them.
 cudaError_t launch_bwd_dq(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tdo,
                           const CUtensorMap& tk, const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L,
-                          KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream) {
+                          KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream,
+                          const BwdLink& link) {
   if (packed) {
     if (d == 64)
       return launch_bwd_impl<64, false, true, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms, nullptr,
-                                                     L, stream);
+                                                     L, stream, link);
     return launch_bwd_impl<128, false, true, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms, nullptr,
-                                                    L, stream);
+                                                    L, stream, link);
   }
   if (f32out) {
     if (d == 64)
       return launch_bwd_impl<64, false, false, true>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms,
-                                                     fill_lengths, L, stream);
+                                                     fill_lengths, L, stream, link);
     return launch_bwd_impl<128, false, false, true>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms,
-                                                    fill_lengths, L, stream);
+                                                    fill_lengths, L, stream, link);
   }
   if (d == 64)
     return launch_bwd_impl<64, false, false, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms,
-                                                    fill_lengths, L, stream);
+                                                    fill_lengths, L, stream, link);
   return launch_bwd_impl<128, false, false, false>(tq, tdo, tk, tv, dq, nullptr, ws, B, H, L, kr, num_sms,
-                                                   fill_lengths, L, stream);
+                                                   fill_lengths, L, stream, link);
 }
 
 // out_rows: rows per (b, h) slice of dK and dV (Lmax, or kr.count for a key
@@ -654,19 +666,20 @@ cudaError_t launch_bwd_dq(int d, bool packed, bool f32out, const CUtensorMap& tq
 // lengths.
 cudaError_t launch_bwd_dkdv(int d, bool packed, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                             const CUtensorMap& tdo, void* dk, void* dv, int* ws, int B, int H, int out_rows, int Lmax,
-                            KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream) {
+                            KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream,
+                            const BwdLink& link) {
   if (packed) {
     if (d == 64)
       return launch_bwd_impl<64, true, true, false>(tk, tv, tq, tdo, dk, dv, ws, B, H, out_rows, kr, num_sms, nullptr,
-                                                    Lmax, stream);
+                                                    Lmax, stream, link);
     return launch_bwd_impl<128, true, true, false>(tk, tv, tq, tdo, dk, dv, ws, B, H, out_rows, kr, num_sms, nullptr,
-                                                   Lmax, stream);
+                                                   Lmax, stream, link);
   }
   if (d == 64)
     return launch_bwd_impl<64, true, false, false>(tk, tv, tq, tdo, dk, dv, ws, B, H, out_rows, kr, num_sms,
-                                                   fill_lengths, Lmax, stream);
+                                                   fill_lengths, Lmax, stream, link);
   return launch_bwd_impl<128, true, false, false>(tk, tv, tq, tdo, dk, dv, ws, B, H, out_rows, kr, num_sms,
-                                                  fill_lengths, Lmax, stream);
+                                                  fill_lengths, Lmax, stream, link);
 }
 
 }  // namespace sigattn

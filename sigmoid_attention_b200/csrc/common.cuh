@@ -52,6 +52,23 @@ struct KeyRange {
   int begin, count;
 };
 
+// How a backward kernel is tied to the kernels around it: `err` receives the
+// error words (nullptr: the header of the kernel's own plan), and `overlap`
+// runs the dK/dV kernel of a whole-backward call beside the dQ kernel
+// launched before it (see bwd.cu).
+struct BwdLink {
+  int* err = nullptr;
+  bool overlap = false;
+};
+
+// One work list that the plan kernel builds: its kind, key range and
+// workspace region (header and list).
+struct PlanRegion {
+  int kind;
+  KeyRange kr;
+  int* ws;
+};
+
 // Valid keys of a sequence of n tokens inside the range.
 __host__ __device__ inline int range_keys(int n, KeyRange kr) {
   return n - kr.begin < 0 ? 0 : (n - kr.begin > kr.count ? kr.count : n - kr.begin);
@@ -285,7 +302,7 @@ __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, flo
       const uint64_t q = f2_mul(t, w);
       const float2 qq = f2_unpack(q);
       if (SLOPE) {
-        const float2 sl = f2_unpack(f2_mul(q, f2_fma(q, f2_splat(-1.0f), f2_splat(1.0f))));  // q (1 - q)
+        const float2 sl = f2_unpack(f2_fma(q ^ 0x8000000080000000ull, q, q));  // q - q^2 = q (1 - q)
         slope[2 * e] = sl.x;
         slope[2 * e + 1] = sl.y;
       }

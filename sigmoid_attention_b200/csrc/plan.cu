@@ -37,12 +37,22 @@ namespace sigattn {
 // is given, from cumulative offsets: sequence b holds packed tokens
 // [cu[b], cu[b+1]), which must lie inside [0, total_tokens]. A sequence that breaks
 // its bounds gets no work items and raises SIGATTN_ERR_INVALID_ARG.
+// One CTA per work list: CTA i builds list `lists[i]` (a whole-backward call
+// builds the dQ and the dK/dV lists at once); length errors go to `err`.
+struct PlanLists {
+  PlanRegion list[2];
+};
+
 __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ lengths, const int* __restrict__ cu,
-                                                    int total_tokens, int B, int H, int L, int kind, KeyRange kr,
-                                                    int* __restrict__ ws) {
+                                                    int total_tokens, int B, int H, int L, PlanLists lists,
+                                                    int* __restrict__ err) {
   // The compute kernel that follows may set itself up meanwhile; it waits
   // for this grid before it reads the plan.
   grid_dep_launch();
+  const PlanRegion region = lists.list[blockIdx.x];
+  const int kind = region.kind;
+  const KeyRange kr = region.kr;
+  int* __restrict__ ws = region.ws;
   extern __shared__ int smem_plan[];
   const int tid = threadIdx.x;
   const int rows = item_rows(kind);
@@ -64,8 +74,8 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
       bad = n < 0 || n > L;
     }
     if (bad) {
-      atomicCAS(ws + kHdrError, 0, 1 /* SIGATTN_ERR_INVALID_ARG */);
-      atomicExch(ws + kHdrErrorSite, -(b + 1));
+      atomicCAS(err + kHdrError, 0, 1 /* SIGATTN_ERR_INVALID_ARG */);
+      atomicExch(err + kHdrErrorSite, -(b + 1));
     }
     s_len[b] = bad ? 0 : n;
     s_start[b] = bad ? 0 : start;
@@ -124,17 +134,38 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
   }
 }
 
-cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, KeyRange kr,
-                        int* ws, cudaStream_t stream) {
-  const int smem = (5 * B + 1) * static_cast<int>(sizeof(int));
+// The plan kernel's shared memory (5 B + 1 ints) may exceed the default
+// 48 KB for large batches: raise its limit once per device.
+static cudaError_t prep_setup() {
   static PerDeviceOnce attr;
-  const cudaError_t e = attr.run([] {
+  return attr.run([] {
     return cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (5 * kMaxBatch + 1) * static_cast<int>(sizeof(int)));
   });
+}
+
+cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int H, int L, int kind, KeyRange kr,
+                        int* ws, cudaStream_t stream) {
+  const cudaError_t e = prep_setup();
   if (e != cudaSuccess) return e;
+  const int smem = (5 * B + 1) * static_cast<int>(sizeof(int));
   const int threads = B <= 256 ? 256 : 1024;
-  prep_kernel<<<1, threads, smem, stream>>>(lengths, cu, total, B, H, L, kind, kr, ws);
+  PlanLists lists{{PlanRegion{kind, kr, ws}, PlanRegion{kind, kr, ws}}};
+  prep_kernel<<<1, threads, smem, stream>>>(lengths, cu, total, B, H, L, lists, ws);
+  return cudaGetLastError();
+}
+
+// The dQ and dK/dV lists of a whole-backward call (padded layout, whole
+// sequences) in one launch: the dQ list in ws_dq, the dK/dV list in ws_dkdv;
+// errors go to ws_dq's header.
+cudaError_t launch_prep_bwd(const int* lengths, int B, int H, int L, int* ws_dq, int* ws_dkdv, cudaStream_t stream) {
+  const cudaError_t e = prep_setup();
+  if (e != cudaSuccess) return e;
+  const int smem = (5 * B + 1) * static_cast<int>(sizeof(int));
+  const int threads = B <= 256 ? 256 : 1024;
+  const KeyRange all{0, L};
+  PlanLists lists{{PlanRegion{kKindDq, all, ws_dq}, PlanRegion{kKindDkdv, all, ws_dkdv}}};
+  prep_kernel<<<2, threads, smem, stream>>>(lengths, nullptr, 0, B, H, L, lists, ws_dq);
   return cudaGetLastError();
 }
 

@@ -42,6 +42,10 @@ def test_status_strings_and_sizes():
     assert sa.sigattn_workspace_size(1, 1, 1, 96) == 0      # unsupported head size
     assert sa.sigattn_workspace_size(0, 1, 1, 64) == 0
     assert sa.sigattn_workspace_size(5000, 1, 1, 64) == 0   # beyond SIGATTN_MAX_BATCH
+    # the whole-backward call holds two work lists, each rounded up to 256 bytes
+    assert sa.sigattn_bwd_workspace_size(4, 16, 4096, 128) == 2 * (256 + 16 * 4 * 16 * 32)
+    assert sa.sigattn_bwd_workspace_size(2, 2, 64, 64) == 2 * 512
+    assert sa.sigattn_bwd_workspace_size(1, 1, 1, 96) == 0
 
 
 def test_bad_arguments_rejected_before_any_device_work():
@@ -54,9 +58,15 @@ def test_bad_arguments_rejected_before_any_device_work():
     assert lib.sigattn_fwd(null, null, null, null, null, 1, 1, 64, 64, null, 0, null) == 1
     assert lib.sigattn_bwd_dq(null, null, null, null, null, null, 1, 1, 64, 64, null, 0, null) == 1
     assert lib.sigattn_bwd_dkdv(null, null, null, null, null, null, null, 1, 1, 64, 64, null, 0, null) == 1
+    assert lib.sigattn_bwd(null, null, null, null, null, null, null, null, 1, 1, 64, 64, null, 0, null) == 1
+    assert lib.sigattn_bwd(null, null, null, null, null, null, null, null, 1, 1, 64, 96, null, 0, null) == 2
     # workspace too small
     lens = (ctypes.c_int * 1)(64)
     assert lib.sigattn_fwd(null, null, null, null, lens, 1, 1, 64, 64, ws, 16, null) == 1
+    # enough for one work list but not for the whole-backward call's two
+    one = sa.sigattn_workspace_size(1, 1, 64, 64)
+    assert one < sa.sigattn_bwd_workspace_size(1, 1, 64, 64)
+    assert lib.sigattn_bwd(null, null, null, null, null, null, null, lens, 1, 1, 64, 64, ws, one, null) == 1
     # negative sizes
     assert lib.sigattn_fwd(null, null, null, null, lens, -1, 1, 64, 64, ws, 4096, null) == 1
     assert lib.sigattn_plan(lens, 1, 1, 64, 64, 7, ws, 4096, null) == 1
