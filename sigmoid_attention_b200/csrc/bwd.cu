@@ -34,8 +34,8 @@
 // leave room in the 512 TMEM columns only for 64-column S and dP regions:
 //   XS [0,BN) XdP [BN,2BN) P [2BN,2.5BN) dS [2.5BN,3BN) A1 [3BN,3BN+D) A2 after.
 // Warps: 0 .. E-1 epilogue, E = 4 G with G column groups (warps 4g..4g+3 take
-// columns [g BN/G, (g+1) BN/G) of each block, in chunks of CW columns; G = 2,
-// CW = 32), then the TMA
+// columns [g BN/G, (g+1) BN/G) of each block, in chunks of CW = 32 columns;
+// G = 4, or 2 for dK/dV at D = 128), then the TMA
 // producer (also claims the work items and passes them on through the
 // shared-memory item ring; for dQ at D = 64 over padded inputs it also writes
 // the zeros of the rows no item covers, with bulk copies from shared memory
@@ -50,11 +50,11 @@ template <int D, bool KV>
 struct BwdCfg {
   static constexpr int BM = kBwdItemRows;   // 128 rows per item
   static constexpr int BN = bwd_col_block(KV, D);
-  // Epilogue column groups (warps per lane quadrant) and chunk width: 8
-  // epilogue warps on 32-column chunks, 16 for dQ at D = 64. (16 warps on
-  // 16-column chunks for dK/dV at D = 128, at 88 registers each, measured
-  // slower: 0.918 -> 0.984 ms on the dense d = 128 workload.)
-  static constexpr int GROUPS = (D == 64) ? 4 : 2;
+  // Epilogue column groups (warps per lane quadrant) and chunk width: 16
+  // epilogue warps on 32-column chunks, except dK/dV at D = 128 (8 warps:
+  // its 64-column blocks would leave 16 warps 16-column chunks, measured
+  // slower: 0.918 -> 0.984 ms on the dense d = 128 workload).
+  static constexpr int GROUPS = (D == 64 || !KV) ? 4 : 2;
   static constexpr int CW = 32;
   static constexpr int NCH = BN / CW;       // chunks per block
   static constexpr int CPW = NCH / GROUPS;  // chunks per epilogue warp
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
             mask_scores(sv[c], valid - CW * c, row_ok);
-            sigmoid_n<true>(sv[c], scale_l2e, neg_log2n, sp[c]);
+            sigmoid_n<true, CW, !KV>(sv[c], scale_l2e, neg_log2n, sp[c]);
             if (KV) {
 #pragma unroll
               for (int e = 0; e < CW / 2; ++e)
@@ -308,10 +308,17 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const uint32_t(&dpc)[CW] = dp[c];
           uint32_t dk[CW / 2];
 #pragma unroll
+          // dS = dP sigma': packed multiplies in the dQ kernel; the dK/dV
+          // kernel, at fewer registers, measured faster with scalar ones.
           for (int e = 0; e < CW / 2; ++e) {
-            const float2 ds = f2_unpack(f2_mul(f2_pack(__uint_as_float(dpc[2 * e]), __uint_as_float(dpc[2 * e + 1])),
-                                               f2_pack(sp[c][2 * e], sp[c][2 * e + 1])));
-            dk[e] = pack_bf16x2(ds.x, ds.y);
+            if constexpr (KV) {
+              dk[e] = pack_bf16x2(__uint_as_float(dpc[2 * e]) * sp[c][2 * e],
+                                  __uint_as_float(dpc[2 * e + 1]) * sp[c][2 * e + 1]);
+            } else {
+              const float2 ds = f2_unpack(f2_mul(f2_pack(__uint_as_float(dpc[2 * e]), __uint_as_float(dpc[2 * e + 1])),
+                                                 f2_pack(sp[c][2 * e], sp[c][2 * e + 1])));
+              dk[e] = pack_bf16x2(ds.x, ds.y);
+            }
           }
           tmem_st(tmem + lane_off + C::TM_DS + (g * CPW + c) * (CW / 2), dk);
           tmem_st_wait();

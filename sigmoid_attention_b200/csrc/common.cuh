@@ -281,7 +281,7 @@ constexpr float kTailC = 0.0625f;
 // about a thousand: the bias -ln n puts the typical weight near 1/n), the
 // short tail form serves; otherwise the general form. Pairs of columns
 // (2e, 2e + 1) go through the packed fp32x2 FMAs.
-template <bool SLOPE, int N>
+template <bool SLOPE, int N, bool SLOPE_FMA = true>
 __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, float neg_log2n, float* slope) {
   static_assert(N == 16 || N == 32, "16 or 32 scores per thread");
   const uint64_t c1 = f2_splat(scale_l2e), c0 = f2_splat(neg_log2n - kTailY);
@@ -302,7 +302,10 @@ __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, flo
       const uint64_t q = f2_mul(t, w);
       const float2 qq = f2_unpack(q);
       if (SLOPE) {
-        const float2 sl = f2_unpack(f2_fma(q ^ 0x8000000080000000ull, q, q));  // q - q^2 = q (1 - q)
+        // q (1 - q): as q - q^2 in one packed FMA, or (SLOPE_FMA false) as
+        // two operations, which the dK/dV epilogue schedules better
+        const float2 sl = SLOPE_FMA ? f2_unpack(f2_fma(q ^ 0x8000000080000000ull, q, q))
+                                    : f2_unpack(f2_mul(q, f2_fma(q, f2_splat(-1.0f), f2_splat(1.0f))));
         slope[2 * e] = sl.x;
         slope[2 * e + 1] = sl.y;
       }
