@@ -587,8 +587,7 @@ def run_gpu(args, w):
             oc, dqc, dkc, dvc = (t[r0:r1] for t in dev_out)
             if packed:
                 sa.sigattn_fwd_varlen(qc, kc, vc, oc, cu_d[c], max_seqlen, ws, stream)
-                sa.sigattn_bwd_dq_varlen(qc, kc, vc, dc, dqc, cu_d[c], max_seqlen, ws, stream)
-                sa.sigattn_bwd_dkdv_varlen(qc, kc, vc, dc, dkc, dvc, cu_d[c], max_seqlen, ws, stream)
+                sa.sigattn_bwd_varlen(qc, kc, vc, dc, dqc, dkc, dvc, cu_d[c], max_seqlen, ws, stream)
             else:
                 lc = lens[r0:r1]
                 sa.sigattn_fwd(qc, kc, vc, oc, lc, ws, stream)
@@ -667,7 +666,7 @@ def run_gpu(args, w):
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps,
                 "schedule": f"{len(rows)} chunks of whole sequences; host-to-device copies, the calls "
-                            f"({'three varlen calls' if packed else 'sigattn_fwd + sigattn_bwd'}) and "
+                            f"({'sigattn_fwd_varlen + sigattn_bwd_varlen' if packed else 'sigattn_fwd + sigattn_bwd'}) and "
                             "device-to-host copies on three streams",
                 "pcie_gbs": pcie, "bound": e2e_bound, "frac_of_bound": e2e_value / e2e_bound,
                 "bound_source": "larger copy direction per step at the measured both-ways pinned copy rate"},

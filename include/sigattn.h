@@ -131,6 +131,11 @@ SIGATTN_API size_t sigattn_bwd_workspace_size(int B, int H, int Lmax, int d);
 SIGATTN_API int sigattn_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
                             void* dv, const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace,
                             size_t workspace_bytes, void* stream);
+/* The same for the packed layout (arguments as sigattn_bwd_dq_varlen; the
+ * workspace is sigattn_bwd_workspace_size(B, H, max_seqlen, d) bytes). */
+SIGATTN_API int sigattn_bwd_varlen(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
+                                   void* dv, const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total,
+                                   int d, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Key ranges: the padded-layout calls restricted to the keys at positions
  * [key_begin, key_begin + key_count) of every sequence, for attention whose

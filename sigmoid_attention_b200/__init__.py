@@ -23,7 +23,7 @@ __all__ = [
     "sigattn_workspace_size", "sigattn_bwd_workspace_size", "sigattn_fwd", "sigattn_fwd_noalloc", "sigattn_bwd",
     "sigattn_bwd_dq", "sigattn_bwd_dkdv", "sigattn_plan",
     "sigattn_plan_host", "sigattn_read_error", "sigattn_last_error", "sigattn_eval_sigmoid", "read_plan", "sigattn_selftest_wait_timeout", "make_workspace", "forward", "backward",
-    "sigattn_fwd_varlen", "sigattn_bwd_dq_varlen", "sigattn_bwd_dkdv_varlen",
+    "sigattn_fwd_varlen", "sigattn_bwd_varlen", "sigattn_bwd_dq_varlen", "sigattn_bwd_dkdv_varlen",
     "sigattn_fwd_partial", "sigattn_bwd_dq_partial", "sigattn_bwd_dkdv_range", "sigattn_cast_bf16",
     "sigattn_softmax_fwd",
     "KIND_FWD", "KIND_DQ", "KIND_DKDV", "SigmoidAttentionFunction", "sigmoid_attention",
@@ -84,6 +84,8 @@ def library():
         lib.sigattn_bwd_dq_varlen.argtypes = [_vp] * 6 + [_i] * 5 + [_vp, _sz, _vp]
         lib.sigattn_bwd_dkdv_varlen.restype = _i
         lib.sigattn_bwd_dkdv_varlen.argtypes = [_vp] * 7 + [_i] * 5 + [_vp, _sz, _vp]
+        lib.sigattn_bwd_varlen.restype = _i
+        lib.sigattn_bwd_varlen.argtypes = [_vp] * 8 + [_i] * 5 + [_vp, _sz, _vp]
         lib.sigattn_plan.restype = _i
         lib.sigattn_plan.argtypes = [_vp] + [_i] * 5 + [_vp, _sz, _vp]
         lib.sigattn_plan_host.restype = _i
@@ -278,6 +280,16 @@ def sigattn_bwd_dq_varlen(q, k, v, dout, dq, cu_seqlens, max_seqlen: int, worksp
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
 
 
+def sigattn_bwd_varlen(q, k, v, dout, dq, dk, dv, cu_seqlens, max_seqlen: int, workspace, stream=None) -> None:
+    """Packed-layout counterpart of sigattn_bwd."""
+    total, H, d = _packed_dims(q)
+    B = cu_seqlens.numel() - 1
+    _check("sigattn_bwd_varlen", library().sigattn_bwd_varlen(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"),
+        _dev(dv, "dv"), _dev(cu_seqlens, "cu_seqlens", torch.int32), B, H, int(max_seqlen), total, d,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_ptr(stream)))
+
+
 def sigattn_bwd_dkdv_varlen(q, k, v, dout, dk, dv, cu_seqlens, max_seqlen: int, workspace, stream=None) -> None:
     total, H, d = _packed_dims(q)
     B = cu_seqlens.numel() - 1
@@ -430,8 +442,7 @@ class SigmoidAttentionVarlenFunction(torch.autograd.Function):
         q, k, v, cu_seqlens, ws = ctx.saved_tensors
         do = do.contiguous()
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        sigattn_bwd_dq_varlen(q, k, v, do, dq, cu_seqlens, ctx.max_seqlen, ws)
-        sigattn_bwd_dkdv_varlen(q, k, v, do, dk, dv, cu_seqlens, ctx.max_seqlen, ws)
+        sigattn_bwd_varlen(q, k, v, do, dq, dk, dv, cu_seqlens, ctx.max_seqlen, ws)
         _check_device_status("sigattn_bwd_varlen", ws, ctx.check)
         return dq, dk, dv, None, None, None
 

@@ -26,7 +26,8 @@ cudaError_t launch_fwd(int d, bool packed, bool f32out, const CUtensorMap& tq, c
                        cudaStream_t stream);
 cudaError_t launch_softmax_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o, int* ws,
                                int B, int H, int L, int num_sms, cudaStream_t stream);
-cudaError_t launch_prep_bwd(const int* lengths, int B, int H, int L, int* ws_dq, int* ws_dkdv, cudaStream_t stream);
+cudaError_t launch_prep_bwd(const int* lengths, const int* cu, int total, int B, int H, int L, int* ws_dq,
+                            int* ws_dkdv, cudaStream_t stream);
 cudaError_t launch_bwd_dq(int d, bool packed, bool f32out, const CUtensorMap& tq, const CUtensorMap& tdo,
                           const CUtensorMap& tk, const CUtensorMap& tv, void* dq, int* ws, int B, int H, int L,
                           KeyRange kr, int num_sms, const int* fill_lengths, cudaStream_t stream,
@@ -266,35 +267,43 @@ size_t plan_region_bytes(int B, int H, int Lmax) {
 // the workspace's first region, dK/dV's in the second), then the dQ kernel
 // and the dK/dV kernel, which takes SMs as the dQ kernel's CTAs finish and
 // completes after it (bwd.cu). Errors of both go to the first header.
-int bwd_padded(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk, void* dv,
-               const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes,
-               void* stream) {
-  if (workspace_bytes < sigattn_bwd_workspace_size(B, H, Lmax, d)) return SIGATTN_ERR_INVALID_ARG;
+// Padded layout: lengths, L = Lmax; packed: cu_seqlens, L = max_seqlen and
+// `total` tokens.
+int bwd_whole(bool packed, const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
+              void* dv, const int32_t* lengths_or_cu, int B, int H, int L, int total, int d, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  if (workspace_bytes < sigattn_bwd_workspace_size(B, H, L, d)) return SIGATTN_ERR_INVALID_ARG;
   DeviceInfo info;
-  int st = check_call(B, H, Lmax, d, lengths, workspace, workspace_bytes, &info);
+  int st = check_call(B, H, L, d, lengths_or_cu, workspace, workspace_bytes, &info);
   if (st != SIGATTN_OK) return st;
+  if (packed && (total < 1 || total > kMaxPackedTokens))
+    return total < 1 ? SIGATTN_ERR_INVALID_ARG : SIGATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
       !aligned16(dv))
     return SIGATTN_ERR_INVALID_ARG;
   const int cb = bwd_col_block(true, d);
+  auto map = [&](CUtensorMap* m, const void* p, int box_rows) {
+    return packed ? make_map_packed(m, p, total, H, d, box_rows) : make_map(m, p, B * H, L, d, box_rows);
+  };
   CUtensorMap tq, tk, tv, tdo, tq_c, tdo_c;
-  if (!make_map(&tq, q, B * H, Lmax, d) || !make_map(&tk, k, B * H, Lmax, d) || !make_map(&tv, v, B * H, Lmax, d) ||
-      !make_map(&tdo, dout, B * H, Lmax, d) || !make_map(&tq_c, q, B * H, Lmax, d, cb) ||
-      !make_map(&tdo_c, dout, B * H, Lmax, d, cb))
+  if (!map(&tq, q, 128) || !map(&tk, k, 128) || !map(&tv, v, 128) || !map(&tdo, dout, 128) || !map(&tq_c, q, cb) ||
+      !map(&tdo_c, dout, cb))
     return map_failure();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws_dq = static_cast<int*>(workspace);
-  int* ws_dkdv = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan_region_bytes(B, H, Lmax));
-  const KeyRange all{0, Lmax};
-  st = cuda_status(launch_prep_bwd(lengths, B, H, Lmax, ws_dq, ws_dkdv, s));
+  int* ws_dkdv = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + plan_region_bytes(B, H, L));
+  const KeyRange all{0, L};
+  const int32_t* lengths = packed ? nullptr : lengths_or_cu;
+  st = cuda_status(launch_prep_bwd(lengths, packed ? lengths_or_cu : nullptr, packed ? total : 0, B, H, L, ws_dq,
+                                   ws_dkdv, s));
   if (st == SIGATTN_OK)
-    st = cuda_status(launch_bwd_dq(d, false, false, tq, tdo, tk, tv, dq, ws_dq, B, H, Lmax, all, info.num_sms,
+    st = cuda_status(launch_bwd_dq(d, packed, false, tq, tdo, tk, tv, dq, ws_dq, B, H, L, all, info.num_sms,
                                    lengths, s));
   if (st != SIGATTN_OK) return st;
   BwdLink link;
   link.err = ws_dq;
   link.overlap = true;
-  return cuda_status(launch_bwd_dkdv(d, false, tk, tv, tq_c, tdo_c, dk, dv, ws_dkdv, B, H, Lmax, Lmax, all,
+  return cuda_status(launch_bwd_dkdv(d, packed, tk, tv, tq_c, tdo_c, dk, dv, ws_dkdv, B, H, L, L, all,
                                      info.num_sms, lengths, s, link));
 }
 
@@ -358,7 +367,14 @@ size_t sigattn_bwd_workspace_size(int B, int H, int Lmax, int d) {
 int sigattn_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk, void* dv,
                 const int32_t* lengths, int B, int H, int Lmax, int d, void* workspace, size_t workspace_bytes,
                 void* stream) {
-  return bwd_padded(q, k, v, dout, dq, dk, dv, lengths, B, H, Lmax, d, workspace, workspace_bytes, stream);
+  return bwd_whole(false, q, k, v, dout, dq, dk, dv, lengths, B, H, Lmax, 0, d, workspace, workspace_bytes, stream);
+}
+
+int sigattn_bwd_varlen(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk, void* dv,
+                       const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total, int d, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return bwd_whole(true, q, k, v, dout, dq, dk, dv, cu_seqlens, B, H, max_seqlen, total, d, workspace,
+                   workspace_bytes, stream);
 }
 
 int sigattn_fwd(const void* q, const void* k, const void* v, void* o, const int32_t* lengths, int B, int H,

@@ -155,17 +155,18 @@ cudaError_t launch_prep(const int* lengths, const int* cu, int total, int B, int
   return cudaGetLastError();
 }
 
-// The dQ and dK/dV lists of a whole-backward call (padded layout, whole
-// sequences) in one launch: the dQ list in ws_dq, the dK/dV list in ws_dkdv;
-// errors go to ws_dq's header.
-cudaError_t launch_prep_bwd(const int* lengths, int B, int H, int L, int* ws_dq, int* ws_dkdv, cudaStream_t stream) {
+// The dQ and dK/dV lists of a whole-backward call (whole sequences, padded
+// layout from `lengths` or packed from `cu` as in launch_prep) in one launch:
+// the dQ list in ws_dq, the dK/dV list in ws_dkdv; errors go to ws_dq's header.
+cudaError_t launch_prep_bwd(const int* lengths, const int* cu, int total, int B, int H, int L, int* ws_dq,
+                            int* ws_dkdv, cudaStream_t stream) {
   const cudaError_t e = prep_setup();
   if (e != cudaSuccess) return e;
   const int smem = (5 * B + 1) * static_cast<int>(sizeof(int));
   const int threads = B <= 256 ? 256 : 1024;
   const KeyRange all{0, L};
   PlanLists lists{{PlanRegion{kKindDq, all, ws_dq}, PlanRegion{kKindDkdv, all, ws_dkdv}}};
-  prep_kernel<<<2, threads, smem, stream>>>(lengths, nullptr, 0, B, H, L, lists, ws_dq);
+  prep_kernel<<<2, threads, smem, stream>>>(lengths, cu, total, B, H, L, lists, ws_dq);
   return cudaGetLastError();
 }
 

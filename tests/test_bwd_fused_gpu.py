@@ -112,3 +112,29 @@ def test_fused_reports_bad_length_in_the_first_header():
     for t in out:  # the bad sequence is treated as empty: all its rows are zero
         assert torch.equal(t[1], torch.zeros_like(t[1]))
         assert torch.isfinite(t[0].float()).all()
+
+
+@pytest.mark.parametrize("name", ["long_8k", "scrna_ragged"])
+def test_fused_varlen_equals_separate_varlen_and_padded(name):
+    # the packed layout: the whole-backward call equals the two packed calls and
+    # the padded whole-backward call on the same sequences, bit for bit
+    w = workloads.WORKLOADS[name]
+    q, k, v, dout, lens = workloads.workload_inputs(w)
+    dev = torch.device("cuda")
+    n = lens.tolist()
+    pack = lambda t: torch.cat([t[b, :, :nb].permute(1, 0, 2) for b, nb in enumerate(n)]).contiguous().to(dev)
+    qp, kp, vp, dp = (pack(t) for t in (q, k, v, dout))
+    cu = torch.tensor([0] + list(np.cumsum(n)), dtype=torch.int32, device=dev)
+    ws = sa.make_workspace(w.B, w.H, max(n), w.d, dev)
+    sep = [torch.full_like(qp, float("nan")) for _ in range(3)]
+    sa.sigattn_bwd_dq_varlen(qp, kp, vp, dp, sep[0], cu, max(n), ws)
+    sa.sigattn_bwd_dkdv_varlen(qp, kp, vp, dp, sep[1], sep[2], cu, max(n), ws)
+    fused = [torch.full_like(qp, float("nan")) for _ in range(3)]
+    sa.sigattn_bwd_varlen(qp, kp, vp, dp, *fused, cu, max(n), ws)
+    assert sa.sigattn_read_error(ws) == (0, 0)
+    for label, a, b in zip(("dq", "dk", "dv"), sep, fused):
+        assert torch.equal(a, b), label
+    _, padded = _separate_and_fused(q, k, v, dout, lens.numpy())
+    for label, a, b in zip(("dq", "dk", "dv"), padded, fused):
+        assert torch.equal(pack(a.cpu()), b), label
+

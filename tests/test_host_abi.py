@@ -60,6 +60,8 @@ def test_bad_arguments_rejected_before_any_device_work():
     assert lib.sigattn_bwd_dkdv(null, null, null, null, null, null, null, 1, 1, 64, 64, null, 0, null) == 1
     assert lib.sigattn_bwd(null, null, null, null, null, null, null, null, 1, 1, 64, 64, null, 0, null) == 1
     assert lib.sigattn_bwd(null, null, null, null, null, null, null, null, 1, 1, 64, 96, null, 0, null) == 2
+    assert lib.sigattn_bwd_varlen(null, null, null, null, null, null, null, null, 1, 1, 64, 64, 64, null, 0,
+                                  null) == 1
     # workspace too small
     lens = (ctypes.c_int * 1)(64)
     assert lib.sigattn_fwd(null, null, null, null, lens, 1, 1, 64, 64, ws, 16, null) == 1
