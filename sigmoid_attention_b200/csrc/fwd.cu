@@ -59,7 +59,7 @@ struct FwdCfg {
   static constexpr int TM_O = 256;
   // At D = 64 the 512 TMEM columns leave room for P in its own region (64
   // columns of bf16 pairs per tile) instead of over S, so S(j+1) need not wait
-  // for PV(j), and all 16 epilogue warps take each tile's sigmoid pass: SEP_P.
+  // for PV(j), and each tile's eight epilogue warps run independently: SEP_P.
   static constexpr bool SEP_P = (D == 64);
   static constexpr int TM_P = TM_O + 2 * D;
   static constexpr int TMEM_COLS = 512;
