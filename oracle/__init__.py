@@ -14,7 +14,8 @@ single-cell Foundation Models" -- sec. 2A (SigmoidAttn equation, bias
 b = -log(n)), sec. 2B (sigma' = sigma(1 - sigma), bounded by 0.25; diagonal
 Jacobian), sec. 2C (padding skipped on both sides; dQ and dK/dV gradients),
 sec. 4A (the softmax comparison; softmax_forward states softmax attention over
-the valid keys, as the attention-survey page writes it).
+the valid keys, as "Transformer Attention機構の効率化と最新派生モデル" writes it
+in its "Vanilla Self-Attention" pseudo code example).
 """
 from __future__ import annotations
 

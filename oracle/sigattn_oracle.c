@@ -208,7 +208,8 @@ int oracle_tiles(const int* lengths, int B, int H, int L, int block, int* out, i
  * the same scheduler ("Better Models, Faster Training: Sigmoid Attention for
  * single-cell Foundation Models", sec. 4A, compares the sigmoid kernel with
  * softmax attention's FlashAttention-2 at 25% padding; sec. 2A contrasts the
- * two weightings; the attention-survey page states softmax attention). For one
+ * two weightings; "Transformer Attention機構の効率化と最新派生モデル" states
+ * softmax attention in its "Vanilla Self-Attention" pseudo code example). For one
  * (b,h) slice and a valid row i < n, over the valid keys j < n only:
  *
  *   S_ij  = <Q_i, K_j> / sqrt(d)             (no bias: softmax normalises)
