@@ -120,17 +120,32 @@ __global__ void __launch_bounds__(1024) prep_kernel(const int* __restrict__ leng
     ws[kHdrNext] = 0;  // the compute kernel's claim counter
     ws[kHdrFill] = 0;  // the dQ kernel's zero-fill claim counter
   }
+  // Each thread writes one contiguous run of the list: item i of sequence
+  // rank s is (b, h, blk) with (h, blk) = divmod(i - s_off[s], row blocks of
+  // b); the first item of the run is located by a binary search, the others
+  // by counting on, so the run costs no search or division per item.
   int4* items = reinterpret_cast<int4*>(ws + kHeaderWords);
-  for (int i = tid; i < total; i += blockDim.x) {
-    int lo = 0, hi = B - 1;  // find s with s_off[s] <= i < s_off[s + 1]
+  const int per = ceil_div(total, static_cast<int>(blockDim.x));
+  const int first = tid * per, end = min(total, first + per);
+  if (first < end) {
+    int lo = 0, hi = B - 1;  // the last s with s_off[s] <= first (a sequence with items)
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (s_off[mid] <= i) lo = mid; else hi = mid - 1;
+      if (s_off[mid] <= first) lo = mid; else hi = mid - 1;
     }
-    const int b = s_order[lo];
-    const int local = i - s_off[lo];
-    const int nblk = ceil_div(work_rows(kind, s_len[b], kr), rows);
-    items[i] = make_int4(b * H + local / nblk, local % nblk, s_len[b], s_start[b]);
+    int b = s_order[lo];
+    int nblk = ceil_div(work_rows(kind, s_len[b], kr), rows);
+    int h = (first - s_off[lo]) / nblk, blk = (first - s_off[lo]) % nblk;
+    for (int i = first; i < end; ++i) {
+      items[i] = make_int4(b * H + h, blk, s_len[b], s_start[b]);
+      if (++blk < nblk) continue;
+      blk = 0;
+      if (++h < H || i + 1 == end) continue;
+      h = 0;  // on to the next sequence with items
+      do ++lo; while (s_off[lo + 1] == s_off[lo]);
+      b = s_order[lo];
+      nblk = ceil_div(work_rows(kind, s_len[b], kr), rows);
+    }
   }
 }
 
