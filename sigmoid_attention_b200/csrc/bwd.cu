@@ -363,8 +363,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const uint32_t(&dpc)[CW] = dp[c];
           uint32_t dk[CW / 2];
 #pragma unroll
-          // dS = dP sigma': packed multiplies in the dQ kernel; the dK/dV
-          // kernel, at fewer registers, measured faster with scalar ones.
+          // dS = dP sigma': packed multiplies in the dQ kernel (whose sigma'
+          // is negated, so that it writes -dS); the dK/dV kernel, at fewer
+          // registers, measured faster with scalar ones.
           for (int e = 0; e < CW / 2; ++e) {
             if constexpr (KV) {
               dk[e] = pack_bf16x2(__uint_as_float(dpc[2 * e]) * sp[c][2 * e],
@@ -408,7 +409,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         const int c = g + G * i;
         const bool second = c >= D / RW;
         const int col = (second ? c - D / RW : c) * RW;
-        const float mul = (second ? 1.0f : scale) * (valid_row ? 1.0f : 0.0f);
+        // the dQ kernel accumulates -dS K (its sigma' comes negated), so its
+        // accumulator takes -scale
+        const float mul = (second ? 1.0f : (KV ? scale : -scale)) * (valid_row ? 1.0f : 0.0f);
         uint32_t v[RW];
         tmem_ld_async(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v);
         tmem_ld_wait(v);

@@ -280,8 +280,12 @@ constexpr float kTailC = 0.0625f;
 // score of the warp lies in the far tail (the usual case once n is more than
 // about a thousand: the bias -ln n puts the typical weight near 1/n), the
 // short tail form serves; otherwise the general form. Pairs of columns
-// (2e, 2e + 1) go through the packed fp32x2 FMAs.
-template <bool SLOPE, int N, bool SLOPE_FMA = true>
+// (2e, 2e + 1) go through the packed fp32x2 FMAs. NEG_SLOPE: slope[e]
+// receives -sigma' instead (exactly the negation; the tail form then runs its
+// polynomial with negated coefficients, which yields -q with no separate sign
+// flip, and -sigma' = (-q)^2 + (-q) is one packed FMA); a[e] still
+// receives sigma.
+template <bool SLOPE, int N, bool NEG_SLOPE = false>
 __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, float neg_log2n, float* slope) {
   static_assert(N == 16 || N == 32, "16 or 32 scores per thread");
   const uint64_t c1 = f2_splat(scale_l2e), c0 = f2_splat(neg_log2n - kTailY);
@@ -297,20 +301,22 @@ __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, flo
     for (int e = 0; e < N / 2; ++e) {
       const float2 zz = f2_unpack(z[e]);
       const uint64_t w = f2_pack(ex2_approx(zz.x), ex2_approx(zz.y));
-      uint64_t t = f2_fma(w, f2_splat(kTailC * kTailC * kTailC), f2_splat(-kTailC * kTailC));
-      t = f2_fma(t, w, f2_splat(kTailC));
-      const uint64_t q = f2_mul(t, w);
+      constexpr float sg = NEG_SLOPE ? -1.0f : 1.0f;  // the sign of q that comes out
+      uint64_t t = f2_fma(w, f2_splat(sg * kTailC * kTailC * kTailC), f2_splat(-sg * kTailC * kTailC));
+      t = f2_fma(t, w, f2_splat(sg * kTailC));
+      const uint64_t q = f2_mul(t, w);  // sg * sigma
       const float2 qq = f2_unpack(q);
       if (SLOPE) {
-        // q (1 - q): as q - q^2 in one packed FMA, or (SLOPE_FMA false) as
-        // two operations, which the dK/dV epilogue schedules better
-        const float2 sl = SLOPE_FMA ? f2_unpack(f2_fma(q ^ 0x8000000080000000ull, q, q))
+        // NEG_SLOPE: (-q)^2 + (-q) = -(q - q^2) in one packed FMA; otherwise
+        // q (1 - q) in two operations, which the dK/dV epilogue schedules
+        // better than q - q^2 with a sign flip
+        const float2 sl = NEG_SLOPE ? f2_unpack(f2_fma(q, q, q))
                                     : f2_unpack(f2_mul(q, f2_fma(q, f2_splat(-1.0f), f2_splat(1.0f))));
         slope[2 * e] = sl.x;
         slope[2 * e + 1] = sl.y;
       }
-      a[2 * e] = __float_as_uint(qq.x);
-      a[2 * e + 1] = __float_as_uint(qq.y);
+      a[2 * e] = __float_as_uint(sg * qq.x);
+      a[2 * e + 1] = __float_as_uint(sg * qq.y);
     }
   } else {
 #pragma unroll
@@ -322,7 +328,7 @@ __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, flo
       const uint64_t r = f2_fma(t, u, f2_splat(1.0f));
       const float2 qq = f2_unpack(q), rr = f2_unpack(r);
       if (SLOPE) {
-        const float2 sl = f2_unpack(f2_mul(q, r));
+        const float2 sl = f2_unpack(NEG_SLOPE ? f2_mul(f2_mul(q, r), f2_splat(-1.0f)) : f2_mul(q, r));
         slope[2 * e] = sl.x;
         slope[2 * e + 1] = sl.y;
       }
@@ -358,8 +364,8 @@ __device__ __forceinline__ float sigmoid_score(float s, float scale_l2e, float n
   float sl[32];
 #pragma unroll
   for (int e = 0; e < 32; ++e) a[e] = __float_as_uint(s);
-  sigmoid32<true>(a, scale_l2e, neg_log2n, sl);
-  *slope = sl[0];
+  sigmoid_n<true, 32, true>(a, scale_l2e, neg_log2n, sl);  // the dQ kernel's form
+  *slope = -sl[0];
   return __uint_as_float(a[0]);
 }
 
