@@ -62,6 +62,14 @@ struct BwdCfg {
   // path in the dK/dV kernel and at D = 128 made those kernels slower, even
   // where no such block occurs.
   static constexpr bool SKIP_DEAD = (!KV && D == 64);
+  // sigma' carried negated (the tail polynomial run with negated
+  // coefficients, -sigma' = (-q)^2 + (-q) in one packed FMA), so the kernel
+  // accumulates -dS products and scales the first accumulator by -scale: no
+  // sign flip per score. Interleaved runs: 0 %-padded dQ 1.664 -> 1.598 ms and
+  // dK/dV 1.958 -> 1.911 ms, dense_d128 dQ 0.649 -> 0.640 ms; dK/dV at
+  // D = 128, whose P also needs the positive sigma, measured slower with it
+  // (0.917 -> 0.933 ms) and keeps sigma' = q (1 - q).
+  static constexpr bool NEG_SLOPE = (!KV || D == 64);
   static constexpr int CW = 32;
   static constexpr int NCH = BN / CW;       // chunks per block
   static constexpr int CPW = NCH / GROUPS;  // chunks per epilogue warp
@@ -319,7 +327,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
             mask_scores(sv[c], valid - CW * c, row_ok);
-            sigmoid_n<true, CW, !KV>(sv[c], scale_l2e, neg_log2n, sp[c]);
+            sigmoid_n<true, CW, C::NEG_SLOPE>(sv[c], scale_l2e, neg_log2n, sp[c]);
             if (KV) {
 #pragma unroll
               for (int e = 0; e < CW / 2; ++e)
@@ -363,9 +371,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const uint32_t(&dpc)[CW] = dp[c];
           uint32_t dk[CW / 2];
 #pragma unroll
-          // dS = dP sigma': packed multiplies in the dQ kernel (whose sigma'
-          // is negated, so that it writes -dS); the dK/dV kernel, at fewer
-          // registers, measured faster with scalar ones.
+          // dS = dP sigma' (-dS with NEG_SLOPE): packed multiplies in the dQ
+          // kernel; the dK/dV kernel, at fewer registers, measured faster
+          // with scalar ones.
           for (int e = 0; e < CW / 2; ++e) {
             if constexpr (KV) {
               dk[e] = pack_bf16x2(__uint_as_float(dpc[2 * e]) * sp[c][2 * e],
@@ -409,9 +417,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         const int c = g + G * i;
         const bool second = c >= D / RW;
         const int col = (second ? c - D / RW : c) * RW;
-        // the dQ kernel accumulates -dS K (its sigma' comes negated), so its
-        // accumulator takes -scale
-        const float mul = (second ? 1.0f : (KV ? scale : -scale)) * (valid_row ? 1.0f : 0.0f);
+        // with NEG_SLOPE the first accumulator holds -dS K (dQ) or -dS^T Q
+        // (dK), so it takes -scale
+        const float mul = (second ? 1.0f : (C::NEG_SLOPE ? -scale : scale)) * (valid_row ? 1.0f : 0.0f);
         uint32_t v[RW];
         tmem_ld_async(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v);
         tmem_ld_wait(v);
