@@ -417,9 +417,9 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         const int c = g + G * i;
         const bool second = c >= D / RW;
         const int col = (second ? c - D / RW : c) * RW;
-        // with NEG_SLOPE the first accumulator holds -dS K (dQ) or -dS^T Q
-        // (dK), so it takes -scale
-        const float mul = (second ? 1.0f : (C::NEG_SLOPE ? -scale : scale)) * (valid_row ? 1.0f : 0.0f);
+        // with NEG_SLOPE the accumulators hold -dS K (dQ), or -dS^T Q and
+        // -P^T dO (dK, dV): they take -scale and -1
+        const float mul = (second ? 1.0f : scale) * (C::NEG_SLOPE ? -1.0f : 1.0f) * (valid_row ? 1.0f : 0.0f);
         uint32_t v[RW];
         tmem_ld_async(tmem + lane_off + (second ? C::TM_A2 : C::TM_A1) + col, v);
         tmem_ld_wait(v);

@@ -283,8 +283,8 @@ constexpr float kTailC = 0.0625f;
 // (2e, 2e + 1) go through the packed fp32x2 FMAs. NEG_SLOPE: slope[e]
 // receives -sigma' instead (exactly the negation; the tail form then runs its
 // polynomial with negated coefficients, which yields -q with no separate sign
-// flip, and -sigma' = (-q)^2 + (-q) is one packed FMA); a[e] still
-// receives sigma.
+// flip, and -sigma' = (-q)^2 + (-q) is one packed FMA), and a[e] receives
+// -sigma.
 template <bool SLOPE, int N, bool NEG_SLOPE = false>
 __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, float neg_log2n, float* slope) {
   static_assert(N == 16 || N == 32, "16 or 32 scores per thread");
@@ -315,8 +315,8 @@ __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, flo
         slope[2 * e] = sl.x;
         slope[2 * e + 1] = sl.y;
       }
-      a[2 * e] = __float_as_uint(sg * qq.x);
-      a[2 * e + 1] = __float_as_uint(sg * qq.y);
+      a[2 * e] = __float_as_uint(qq.x);  // sg * sigma
+      a[2 * e + 1] = __float_as_uint(qq.y);
     }
   } else {
 #pragma unroll
@@ -332,8 +332,9 @@ __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, flo
         slope[2 * e] = sl.x;
         slope[2 * e + 1] = sl.y;
       }
-      a[2 * e] = __float_as_uint(yy.x < 0.0f ? qq.x : rr.x);
-      a[2 * e + 1] = __float_as_uint(yy.y < 0.0f ? qq.y : rr.y);
+      constexpr float sg = NEG_SLOPE ? -1.0f : 1.0f;
+      a[2 * e] = __float_as_uint(sg * (yy.x < 0.0f ? qq.x : rr.x));
+      a[2 * e + 1] = __float_as_uint(sg * (yy.y < 0.0f ? qq.y : rr.y));
     }
   }
 }
@@ -366,7 +367,7 @@ __device__ __forceinline__ float sigmoid_score(float s, float scale_l2e, float n
   for (int e = 0; e < 32; ++e) a[e] = __float_as_uint(s);
   sigmoid_n<true, 32, true>(a, scale_l2e, neg_log2n, sl);  // the dQ kernel's form
   *slope = -sl[0];
-  return __uint_as_float(a[0]);
+  return -__uint_as_float(a[0]);
 }
 
 // Zero one unit of the output rows that no work item covers: rows
