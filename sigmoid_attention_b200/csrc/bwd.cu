@@ -62,14 +62,14 @@ struct BwdCfg {
   // path in the dK/dV kernel and at D = 128 made those kernels slower, even
   // where no such block occurs.
   static constexpr bool SKIP_DEAD = (!KV && D == 64);
-  // sigma' carried negated (the tail polynomial run with negated
-  // coefficients, -sigma' = (-q)^2 + (-q) in one packed FMA), so the kernel
-  // accumulates -dS products and scales the first accumulator by -scale: no
-  // sign flip per score. Interleaved runs: 0 %-padded dQ 1.664 -> 1.598 ms and
-  // dK/dV 1.958 -> 1.911 ms, dense_d128 dQ 0.649 -> 0.640 ms; dK/dV at
-  // D = 128, whose P also needs the positive sigma, measured slower with it
-  // (0.917 -> 0.933 ms) and keeps sigma' = q (1 - q).
-  static constexpr bool NEG_SLOPE = (!KV || D == 64);
+  // sigma and sigma' are carried negated (the tail polynomial run with
+  // negated coefficients gives -sigma, and -sigma' = (-sigma)^2 + (-sigma) is
+  // one packed FMA), so the kernel writes -P and -dS, its accumulators hold
+  // -dQ / scale, or -dK / scale and -dV, and the readout multiplies by -scale
+  // and -1: no sign flip per score. Interleaved runs: 0 %-padded dQ 1.664 ->
+  // 1.598 ms and dK/dV 1.958 -> 1.853 ms, dense_d128 dQ 0.649 -> 0.640 ms and
+  // dK/dV 0.949 -> 0.936 ms.
+  static constexpr bool NEG_SLOPE = true;
   static constexpr int CW = 32;
   static constexpr int NCH = BN / CW;       // chunks per block
   static constexpr int CPW = NCH / GROUPS;  // chunks per epilogue warp
