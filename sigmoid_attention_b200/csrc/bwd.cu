@@ -371,11 +371,12 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const uint32_t(&dpc)[CW] = dp[c];
           uint32_t dk[CW / 2];
 #pragma unroll
-          // dS = dP sigma' (-dS with NEG_SLOPE): packed multiplies in the dQ
-          // kernel; the dK/dV kernel, at fewer registers, measured faster
-          // with scalar ones.
+          // -dS = dP (-sigma'): packed multiplies, except in the dK/dV kernel
+          // at D = 64 (fewer registers), which measured faster with scalar
+          // ones (0 %-padded 1.853 against 1.861 ms; at D = 128 packed 0.926
+          // against 0.935 ms).
           for (int e = 0; e < CW / 2; ++e) {
-            if constexpr (KV) {
+            if constexpr (KV && D == 64) {
               dk[e] = pack_bf16x2(__uint_as_float(dpc[2 * e]) * sp[c][2 * e],
                                   __uint_as_float(dpc[2 * e + 1]) * sp[c][2 * e + 1]);
             } else {
