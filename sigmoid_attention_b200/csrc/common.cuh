@@ -286,7 +286,8 @@ constexpr float kTailC = 0.0625f;
 // flip, and -sigma' = (-q)^2 + (-q) is one packed FMA), and a[e] receives
 // -sigma.
 template <bool SLOPE, int N, bool NEG_SLOPE = false>
-__device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, float neg_log2n, float* slope) {
+__device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, float neg_log2n, float* slope,
+                                          bool lane_ok = true) {
   static_assert(N == 16 || N == 32, "16 or 32 scores per thread");
   const uint64_t c1 = f2_splat(scale_l2e), c0 = f2_splat(neg_log2n - kTailY);
   uint64_t z[N / 2];  // z = y - kTailY
@@ -296,7 +297,9 @@ __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, flo
     z[e] = f2_fma(f2_pack(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1])), c1, c0);
     all &= static_cast<uint32_t>(z[e]) & static_cast<uint32_t>(z[e] >> 32);
   }
-  if (__all_sync(0xffffffffu, (all >> 31) != 0)) {
+  // Lanes with lane_ok false (rows whose outputs are discarded) take no part
+  // in the choice; what they compute is not meaningful.
+  if (__all_sync(0xffffffffu, (all >> 31) != 0 || !lane_ok)) {
 #pragma unroll
     for (int e = 0; e < N / 2; ++e) {
       const float2 zz = f2_unpack(z[e]);
@@ -340,8 +343,9 @@ __device__ __forceinline__ void sigmoid_n(uint32_t (&a)[N], float scale_l2e, flo
 }
 
 template <bool SLOPE>
-__device__ __forceinline__ void sigmoid32(uint32_t (&a)[32], float scale_l2e, float neg_log2n, float* slope) {
-  sigmoid_n<SLOPE, 32>(a, scale_l2e, neg_log2n, slope);
+__device__ __forceinline__ void sigmoid32(uint32_t (&a)[32], float scale_l2e, float neg_log2n, float* slope,
+                                          bool lane_ok = true) {
+  sigmoid_n<SLOPE, 32>(a, scale_l2e, neg_log2n, slope, lane_ok);
 }
 
 // Scores that must not count: the columns at or past `valid` (keys beyond

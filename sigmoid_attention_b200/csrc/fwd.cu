@@ -534,12 +534,20 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       const float neg_log2n = -__log2f(static_cast<float>(n));  // bias * log2(e)
       const int t = ot;  // this warp's tile; the two tiles' warps run independently
       const int h = oc;  // its 64-column half of each key block (two 32-column chunks)
-      for (int j = 0; ok && t < ntiles && j < nkb; ++j) {
-        if (!(ok = mbar_wait(&bar.s_full[t], sph[t], abort_flag, ws, 121))) break;
+      // A padded row's weights only reach its own output row, which is
+      // discarded: such rows are not masked, and they take no part in the
+      // warp's choice of sigmoid form (so their values never change a valid
+      // output's bits).
+      const bool row_ok = row_base + t * C::BM + r < n;
+      // One pass over key block j. MASKED (the last block, the only one that
+      // can hold keys past the sequence): those scores are set to -inf before
+      // the sigmoid; the other passes carry no masking code at all.
+      auto pass = [&](const int j, auto masked) -> bool {
+        constexpr bool MASKED = decltype(masked)::value;
+        if (!mbar_wait(&bar.s_full[t], sph[t], abort_flag, ws, 121)) return false;
         sph[t] ^= 1;
         for (int i = 0; i < 2; ++i) {
           const int cc = 2 * h + i;
-          const int valid = nk - (j * C::BN + 32 * cc);  // columns < valid are real keys
           tc_fence_after();
           uint32_t a[32];
           tmem_ld32(tmem + lane_off + C::TM_S + t * 128 + 32 * cc, a);
@@ -549,24 +557,28 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
             if (lane == 0) mbar_arrive(&bar.s_read[t]);
           }
           uint32_t pk[16];
-          mask_scores(a, valid, row_base + t * C::BM + r < n);
-          sigmoid32<false>(a, scale_l2e, neg_log2n, nullptr);
+          if constexpr (MASKED) mask_scores(a, nk - (j * C::BN + 32 * cc), true);  // columns < that are keys
+          sigmoid32<false>(a, scale_l2e, neg_log2n, nullptr, row_ok);
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
           // The P region is free once the tile's previous PV products completed.
           if (i == 0 && pv_pending[t]) {
-            if (!(ok = mbar_wait(&bar.pv_done[t], pvph[t], abort_flag, ws, 124))) break;
+            if (!mbar_wait(&bar.pv_done[t], pvph[t], abort_flag, ws, 124)) return false;
             pvph[t] ^= 1;
           }
           pv_pending[t] = true;
           tc_fence_after();
           tmem_st16(tmem + lane_off + C::TM_P + t * 64 + 16 * cc, pk);
         }
-        if (!ok) break;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar.p_full[2 * t + h]);
+        return true;
+      };
+      if (t < ntiles) {
+        for (int j = 0; ok && j + 1 < nkb; ++j) ok = pass(j, std::false_type{});
+        if (ok) ok = pass(nkb - 1, std::true_type{});
       }
       if (!ok) break;
       const int row = row_base + ot * C::BM + r;
