@@ -70,6 +70,12 @@ struct BwdCfg {
   // 1.598 ms and dK/dV 1.958 -> 1.853 ms, dense_d128 dQ 0.649 -> 0.640 ms and
   // dK/dV 0.949 -> 0.936 ms.
   static constexpr bool NEG_SLOPE = true;
+  // Blocks before the last run without masking code (a second instance of
+  // the block's code): dQ 0 %-padded 1.599 -> 1.552 ms, 75 % 0.1647 ->
+  // 0.1602 ms, dense_d128 0.663 -> 0.657 ms; dK/dV at D = 128 0.934 ->
+  // 0.929 ms. The dK/dV kernel at D = 64 spills with two instances (1.854 ->
+  // 1.912 ms) and runs every block in the masking form.
+  static constexpr bool SPLIT_MASK = !(KV && D == 64);
   static constexpr int CW = 32;
   static constexpr int NCH = BN / CW;       // chunks per block
   static constexpr int CPW = NCH / GROUPS;  // chunks per epilogue warp
@@ -260,13 +266,19 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
       // skips such work: elsewhere the extra path measured slower).
       const bool rows_dead = C::SKIP_DEAD && __all_sync(0xffffffffu, !row_ok);
       const float neg_log2n = -__log2f(static_cast<float>(n));  // bias * log2(e)
-      for (int j = 0; j < nb; ++j) {
-        if (C::SKIP_DEAD && (ncols - (j * C::BN + g * CPW * CW) <= 0 || rows_dead)) {
+      // One column block. Padded rows are not masked (their values reach
+      // only their own, discarded output rows, and they take no part in the
+      // choice of sigmoid form); only the last block can hold columns past the
+      // sequence, and with SPLIT_MASK it alone runs the MASKED form, which
+      // sets their scores to -inf before the sigmoid.
+      auto block = [&](const int j, auto masked) -> bool {
+        constexpr bool MASKED = decltype(masked)::value;
+        if (C::SKIP_DEAD && ((MASKED && ncols - (j * C::BN + g * CPW * CW) <= 0) || rows_dead)) {
           // No valid score in this warp's columns of the block (past the
           // sequence's end, or padded rows only): sigma' and dS are all 0.
           // The warp reads neither S nor dP and only keeps its part in the
           // hand-offs, writing zeros.
-          if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, err, 221))) break;
+          if (!mbar_wait(&bar.xs_full, s_ph, abort_flag, err, 221)) return false;
           s_ph ^= 1;
           tc_fence_before();
           __syncwarp();
@@ -275,7 +287,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
 #pragma unroll
           for (int e = 0; e < CW / 2; ++e) zero[e] = 0u;
           if (KV) {
-            if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, err, 223))) break;
+            if (!mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, err, 223)) return false;
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < CPW; ++c) {
@@ -286,14 +298,14 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
               if (lane == 0) mbar_arrive(&bar.p_full[g * CPW + c]);
             }
           }
-          if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, err, 222))) break;
+          if (!mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, err, 222)) return false;
           dp_ph[xb] ^= 1;
           uint64_t* xdp_read = &bar.xdp_read[xb];
           if (++xb == static_cast<uint32_t>(C::NXDP)) xb = 0;
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(xdp_read);
-          if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, err, 224))) break;
+          if (!mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, err, 224)) return false;
           free_ph ^= 1;
           tc_fence_after();
 #pragma unroll
@@ -304,7 +316,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar.ds_full[g * CPW + c]);
           }
-          continue;
+          return true;
         }
         // ---- S -> sigma'(x) = P (1 - P) kept in registers for dS, and (dK/dV)
         // bf16 P for dV, written once the previous block's dV products have
@@ -313,7 +325,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         uint32_t pk[KV ? CPW : 1][CW / 2];
         {
           uint32_t sv[CPW][CW];
-          if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, err, 221))) break;
+          if (!mbar_wait(&bar.xs_full, s_ph, abort_flag, err, 221)) return false;
           s_ph ^= 1;
           tc_fence_after();
 #pragma unroll
@@ -326,8 +338,8 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           const int valid = ncols - (j * C::BN + g * CPW * CW);  // columns < valid are real tokens
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
-            mask_scores(sv[c], valid - CW * c, row_ok);
-            sigmoid_n<true, CW, C::NEG_SLOPE>(sv[c], scale_l2e, neg_log2n, sp[c]);
+            if constexpr (MASKED) mask_scores(sv[c], valid - CW * c, true);
+            sigmoid_n<true, CW, C::NEG_SLOPE>(sv[c], scale_l2e, neg_log2n, sp[c], row_ok);
             if (KV) {
 #pragma unroll
               for (int e = 0; e < CW / 2; ++e)
@@ -336,7 +348,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           }
         }
         if (KV) {
-          if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, err, 223))) break;
+          if (!mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, err, 223)) return false;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
@@ -352,7 +364,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         uint32_t dp[CPW][CW];
         const uint32_t tXDP = xb ? tXDP1 : tXDP0;
         uint64_t* xdp_read = &bar.xdp_read[xb];
-        if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, err, 222))) break;
+        if (!mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, err, 222)) return false;
         dp_ph[xb] ^= 1;
         if (++xb == static_cast<uint32_t>(C::NXDP)) xb = 0;
         tc_fence_after();
@@ -363,7 +375,7 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(xdp_read);
-        if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, err, 224))) break;
+        if (!mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, err, 224)) return false;
         free_ph ^= 1;
         tc_fence_after();
 #pragma unroll
@@ -390,6 +402,147 @@ __global__ void __launch_bounds__(BwdCfg<D, KV>::THREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar.ds_full[g * CPW + c]);
+        }
+        return true;
+      };
+      if constexpr (C::SPLIT_MASK) {
+        for (int j = 0; ok && j + 1 < nb; ++j) ok = block(j, std::false_type{});
+        if (ok) ok = block(nb - 1, std::true_type{});
+      } else {
+        // One form for every block, padded rows and columns masked (the
+        // block's code as one loop body, which keeps this kernel free of
+        // spills).
+        for (int j = 0; j < nb; ++j) {
+          if (C::SKIP_DEAD && (ncols - (j * C::BN + g * CPW * CW) <= 0 || rows_dead)) {
+            // No valid score in this warp's columns of the block (past the
+            // sequence's end, or padded rows only): sigma' and dS are all 0.
+            // The warp reads neither S nor dP and only keeps its part in the
+            // hand-offs, writing zeros.
+            if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, err, 221))) break;
+            s_ph ^= 1;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.xs_read);
+            uint32_t zero[CW / 2];
+  #pragma unroll
+            for (int e = 0; e < CW / 2; ++e) zero[e] = 0u;
+            if (KV) {
+              if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, err, 223))) break;
+              tc_fence_after();
+  #pragma unroll
+              for (int c = 0; c < CPW; ++c) {
+                tmem_st(tmem + lane_off + C::TM_P + (g * CPW + c) * (CW / 2), zero);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar.p_full[g * CPW + c]);
+              }
+            }
+            if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, err, 222))) break;
+            dp_ph[xb] ^= 1;
+            uint64_t* xdp_read = &bar.xdp_read[xb];
+            if (++xb == static_cast<uint32_t>(C::NXDP)) xb = 0;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xdp_read);
+            if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, err, 224))) break;
+            free_ph ^= 1;
+            tc_fence_after();
+  #pragma unroll
+            for (int c = 0; c < CPW; ++c) {
+              tmem_st(tmem + lane_off + C::TM_DS + (g * CPW + c) * (CW / 2), zero);
+              tmem_st_wait();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bar.ds_full[g * CPW + c]);
+            }
+            continue;
+          }
+          // ---- S -> sigma'(x) = P (1 - P) kept in registers for dS, and (dK/dV)
+          // bf16 P for dV, written once the previous block's dV products have
+          // read the P region. Padded columns get P = sigma' = 0.
+          float sp[CPW][CW];
+          uint32_t pk[KV ? CPW : 1][CW / 2];
+          {
+            uint32_t sv[CPW][CW];
+            if (!(ok = mbar_wait(&bar.xs_full, s_ph, abort_flag, err, 221))) break;
+            s_ph ^= 1;
+            tc_fence_after();
+  #pragma unroll
+            for (int c = 0; c < CPW; ++c) tmem_ld_async(tXS + CW * c, sv[c]);
+  #pragma unroll
+            for (int c = 0; c < CPW; ++c) tmem_ld_wait(sv[c]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.xs_read);
+            const int valid = ncols - (j * C::BN + g * CPW * CW);  // columns < valid are real tokens
+  #pragma unroll
+            for (int c = 0; c < CPW; ++c) {
+              mask_scores(sv[c], valid - CW * c, row_ok);
+              sigmoid_n<true, CW, C::NEG_SLOPE>(sv[c], scale_l2e, neg_log2n, sp[c]);
+              if (KV) {
+  #pragma unroll
+                for (int e = 0; e < CW / 2; ++e)
+                  pk[KV ? c : 0][e] = pack_bf16x2(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1]));
+              }
+            }
+          }
+          if (KV) {
+            if (!(ok = mbar_wait(&bar.p_free, free_ph ^ 1, abort_flag, err, 223))) break;
+            tc_fence_after();
+  #pragma unroll
+            for (int c = 0; c < CPW; ++c) {
+              tmem_st(tmem + lane_off + C::TM_P + (g * CPW + c) * (CW / 2), pk[KV ? c : 0]);
+              tmem_st_wait();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bar.p_full[g * CPW + c]);
+            }
+          }
+          // ---- dP -> dS = dP P (1 - P), bf16 dS for dQ / dK: dP is copied out
+          // whole, so its region is released at once.
+          uint32_t dp[CPW][CW];
+          const uint32_t tXDP = xb ? tXDP1 : tXDP0;
+          uint64_t* xdp_read = &bar.xdp_read[xb];
+          if (!(ok = mbar_wait(&bar.xdp_full[xb], dp_ph[xb], abort_flag, err, 222))) break;
+          dp_ph[xb] ^= 1;
+          if (++xb == static_cast<uint32_t>(C::NXDP)) xb = 0;
+          tc_fence_after();
+  #pragma unroll
+          for (int c = 0; c < CPW; ++c) tmem_ld_async(tXDP + CW * c, dp[c]);
+  #pragma unroll
+          for (int c = 0; c < CPW; ++c) tmem_ld_wait(dp[c]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xdp_read);
+          if (!(ok = mbar_wait(&bar.ds_free, free_ph ^ 1, abort_flag, err, 224))) break;
+          free_ph ^= 1;
+          tc_fence_after();
+  #pragma unroll
+          for (int c = 0; c < CPW; ++c) {
+            const uint32_t(&dpc)[CW] = dp[c];
+            uint32_t dk[CW / 2];
+  #pragma unroll
+            // -dS = dP (-sigma'): packed multiplies, except in the dK/dV kernel
+            // at D = 64 (fewer registers), which measured faster with scalar
+            // ones (0 %-padded 1.853 against 1.861 ms; at D = 128 packed 0.926
+            // against 0.935 ms).
+            for (int e = 0; e < CW / 2; ++e) {
+              if constexpr (KV && D == 64) {
+                dk[e] = pack_bf16x2(__uint_as_float(dpc[2 * e]) * sp[c][2 * e],
+                                    __uint_as_float(dpc[2 * e + 1]) * sp[c][2 * e + 1]);
+              } else {
+                const float2 ds = f2_unpack(f2_mul(f2_pack(__uint_as_float(dpc[2 * e]), __uint_as_float(dpc[2 * e + 1])),
+                                                   f2_pack(sp[c][2 * e], sp[c][2 * e + 1])));
+                dk[e] = pack_bf16x2(ds.x, ds.y);
+              }
+            }
+            tmem_st(tmem + lane_off + C::TM_DS + (g * CPW + c) * (CW / 2), dk);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.ds_full[g * CPW + c]);
+          }
         }
       }
       if (!ok) break;

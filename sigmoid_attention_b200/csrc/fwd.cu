@@ -630,17 +630,23 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
       const int nk = range_keys(n, kr);
       const int nkb = ceil_div(nk, C::BN);
       const float neg_log2n = -__log2f(static_cast<float>(n));  // bias * log2(e)
-      for (int j = 0; j < nkb; ++j) {
-        if (!(ok = mbar_wait(&bar.s_full[t], sph, abort_flag, ws, 121))) break;
+      // Padded rows are not masked: their weights reach only their own,
+      // discarded output rows, and they take no part in the choice of
+      // sigmoid form. Only the last block can hold keys past the sequence:
+      // it alone runs the MASKED pass, whose scores of those keys are set to
+      // -inf before the sigmoid.
+      const bool row_ok = row < n;
+      auto pass = [&](const int j, auto masked) -> bool {
+        constexpr bool MASKED = decltype(masked)::value;
+        if (!mbar_wait(&bar.s_full[t], sph, abort_flag, ws, 121)) return false;
         sph ^= 1;
         // Take turns with the other tile (two-tile items only): tile 1 waits
         // for tile 0's pass over block j, tile 0 for tile 1's pass over j-1.
         if (two_tiles && (t == 1 || j > 0)) {
-          if (!(ok = mbar_wait(&bar.epi_done[1 - t], turn_ph, abort_flag, ws, 123))) break;
+          if (!mbar_wait(&bar.epi_done[1 - t], turn_ph, abort_flag, ws, 123)) return false;
           turn_ph ^= 1;
         }
         tc_fence_after();
-        const int valid = nk - (j * C::BN + h * 64);  // columns < valid are real keys
         // The half's 64 keys in two 32-column chunks; P of chunk c goes to
         // TMEM columns [16c, 16c + 16) of the half, which hold S values this
         // thread has already read (chunk 0's).
@@ -649,8 +655,8 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           uint32_t a[32];
           tmem_ld32(tS + 32 * c, a);
           uint32_t pk[16];
-          mask_scores(a, valid - 32 * c, row < n);
-          sigmoid32<false>(a, scale_l2e, neg_log2n, nullptr);
+          if constexpr (MASKED) mask_scores(a, nk - (j * C::BN + h * 64 + 32 * c), true);  // columns < that are keys
+          sigmoid32<false>(a, scale_l2e, neg_log2n, nullptr, row_ok);
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
           tmem_st16(tS + 16 * c, pk);
@@ -664,7 +670,10 @@ __global__ void __launch_bounds__((16 + 3) * 32, 1)
           // tile 1's last pass of the item has no successor to wait for it.
           if (two_tiles && (t == 0 || j + 1 < nkb)) mbar_arrive(&bar.epi_done[t]);
         }
-      }
+        return true;
+      };
+      for (int j = 0; ok && j + 1 < nkb; ++j) ok = pass(j, std::false_type{});
+      if (ok) ok = pass(nkb - 1, std::true_type{});
       if (!ok) break;
       if (!(ok = mbar_wait(&bar.o_full[t], oph, abort_flag, ws, 122))) break;
       oph ^= 1;
