@@ -24,6 +24,9 @@
 //   XdP = R2 C2_j^T  (dP, fp32)  -> epilogue: dS = dP P (1 - P); bf16 dS to
 //                                   its own region
 //   A1 += dS C1_j, A2 += P C2_j  (A operand read from TMEM, per 32-column chunk)
+// (The kernels hold -P and -dS in TMEM and accumulate -dQ / scale, -dK / scale
+// and -dV, and the readout multiplies by -scale and -1: the negated forms come
+// out of the sigmoid's polynomial without a sign flip per score.)
 // A region is released as soon as the epilogue has copied it to registers, so
 // the products of block j+1 overlap the epilogue of block j. One thread issues
 // a tcgen05.mma only every ~100 cycles, so the products are spread over four
