@@ -21,8 +21,10 @@
  *    are zero) and raises SIGATTN_ERR_INVALID_ARG in the workspace's sticky
  *    error word (read it with sigattn_read_error).
  *  - Outputs are fully written: rows i >= n_b of O, dQ, dK and dV are exact
- *    zeros. Values in padded rows of the inputs are never used, but must be
- *    finite: a padded value v enters as 0 * v inside the tensor-core sums.
+ *    zeros. Values in padded rows of the inputs never change an output, but
+ *    must be finite: a padded value v enters a valid result only as 0 * v
+ *    inside the tensor-core sums (the discarded results of padded rows
+ *    themselves may use it).
  *  - The scale is 1/sqrt(d) and the bias -ln(n_b) is computed in-kernel; the
  *    bias has no gradient. There is no causal mask.
  *  - Arithmetic: bf16 operands, fp32 accumulation, P (and dS) rounded to bf16
@@ -207,8 +209,8 @@ SIGATTN_API int sigattn_cast_bf16(const float* x, void* y, long long count, void
  *    [cu_seqlens[b], cu_seqlens[b+1]) are never touched. Results equal those of
  *    the padded calls on the same sequences. The last row block of a sequence
  *    reads up to 255 rows past its end (the next sequence, or rows after
- *    cu_seqlens[B]); those enter only as 0 * value and must be finite, as
- *    padded rows must be in the padded layout.
+ *    cu_seqlens[B]); those enter a result of the sequence only as 0 * value
+ *    and must be finite, as padded rows must be in the padded layout.
  *  - 1 <= total <= INT32_MAX - 4096; workspace: sigattn_workspace_size(B, H,
  *    max_seqlen, d) bytes. Everything else as for the padded calls. */
 SIGATTN_API int sigattn_fwd_varlen(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
